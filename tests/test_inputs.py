@@ -1,0 +1,34 @@
+"""The seeded generators: same seed -> same tensors, documented ranges and dtypes."""
+import torch
+
+from sparse_attention_17_b200 import inputs as G
+
+
+def test_tiny_fp32_ranges_and_determinism():
+    a, b = G.tiny_fp32(T=64), G.tiny_fp32(T=64)
+    for key in ("q_idx", "k_idx", "w", "q", "k", "v"):
+        assert torch.equal(a[key], b[key]) and a[key].dtype == torch.float32
+    assert a["q_idx"].min() >= -8 and a["q_idx"].max() <= 8
+    assert a["w"].min() >= 1 and a["w"].max() <= 4
+    assert torch.equal(a["q_idx"], a["q_idx"].round())
+
+
+def test_mla_int_ranges():
+    d = G.mla_prefill_int(T=128)
+    assert d["q_idx"].dtype == torch.bfloat16 and d["q"].shape == (128, 16, 576)
+    assert d["kv"].shape == (128, 576)
+    assert int(d["q_idx"].float().abs().max()) <= 4 and d["w"].min() >= 1 and d["w"].max() <= 3
+    assert 0.4 < d["kv"].float().std().item() < 0.6
+
+
+def test_decode_pages_are_a_permutation():
+    d = G.mla_decode(B=4, L=300, page_size=64)
+    pt = d["page_table"]
+    assert pt.shape == (4, 5)
+    assert torch.equal(pt.flatten().sort().values, torch.arange(20, dtype=torch.int32))
+
+
+def test_stack_seeds_per_layer():
+    s = G.layer_stack(T=32, pattern="FSS")
+    assert "q_idx" in s["layers"][0] and "q_idx" not in s["layers"][1]
+    assert not torch.equal(s["layers"][0]["q"], s["layers"][1]["q"])
