@@ -60,7 +60,7 @@ def tiny_fp32(T: int = 3072, seed: int = 0, k: int = 512) -> dict:
     d["q"] = _normal(g, 1.0, (T, H_TINY, D_TINY), torch.float32)
     d["k"] = _normal(g, 1.0, (T, H_TINY, D_TINY), torch.float32)
     d["v"] = _normal(g, 1.0, (T, H_TINY, D_TINY), torch.float32)
-    d.update(T=T, k=k, scale=SCALE_TINY)
+    d.update(T=T, topk=k, scale=SCALE_TINY)
     return d
 
 
@@ -91,7 +91,7 @@ def mla_prefill_int(T: int = 8192, seed: int = 0, k: int = 2048) -> dict:
     g = _gen(seed)
     d = indexer_int(T, seed, g=g)
     d.update(mla_layer(T, seed, g=g))
-    d.update(T=T, k=k, scale=SCALE_MLA)
+    d.update(T=T, topk=k, scale=SCALE_MLA)
     return d
 
 
@@ -99,7 +99,7 @@ def mla_prefill_gauss(T: int = 65536, seed: int = 0, k: int = 2048) -> dict:
     g = _gen(seed)
     d = indexer_gauss(T, seed, g=g)
     d.update(mla_layer(T, seed, g=g))
-    d.update(T=T, k=k, scale=SCALE_MLA)
+    d.update(T=T, topk=k, scale=SCALE_MLA)
     return d
 
 
@@ -118,7 +118,7 @@ def layer_stack(T: int = 16384, pattern: str = "FSS" * 9, k: int = 2048,
         if ch == "F":
             L.update(indexer_int(T, indexer_seed_base + l))
         out.append(L)
-    return {"layers": out, "pattern": pattern, "T": T, "k": k, "scale": SCALE_MLA}
+    return {"layers": out, "pattern": pattern, "T": T, "topk": k, "scale": SCALE_MLA}
 
 
 def mla_decode(B: int = 64, L: int = 32768, seed: int = 0, k: int = 2048,
@@ -138,5 +138,5 @@ def mla_decode(B: int = 64, L: int = 32768, seed: int = 0, k: int = 2048,
     if seq_lens is None:
         seq_lens = [L] * B
     d["seq_lens"] = torch.tensor(seq_lens, dtype=torch.int32)
-    d.update(B=B, L=L, k=k, page_size=page_size, scale=SCALE_MLA)
+    d.update(B=B, L=L, topk=k, page_size=page_size, scale=SCALE_MLA)
     return d

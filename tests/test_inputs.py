@@ -10,7 +10,7 @@ def test_tiny_fp32_ranges_and_determinism():
         assert torch.equal(a[key], b[key]) and a[key].dtype == torch.float32
     assert a["q_idx"].min() >= -8 and a["q_idx"].max() <= 8
     assert a["w"].min() >= 1 and a["w"].max() <= 4
-    assert torch.equal(a["q_idx"], a["q_idx"].round())
+    assert torch.equal(a["q_idx"], torch.round(a["q_idx"]))
 
 
 def test_mla_int_ranges():
