@@ -1,0 +1,421 @@
+"""Benchmark of the DSA prefill hot path: lightning indexer -> per-row top-k -> sparse
+absorbed MLA, one layer at T = 65536 with top-2048 (16 indexer heads x 64, 16 query heads,
+576-dim latent), on synthetic seeded inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  With N > 1 (launched by torchrun) every rank runs its own
+independent sequence (weak scaling, no data-path collective); the time is the max over
+ranks.  ``--impl reference`` times the CPU oracle on a bounded sample of query rows.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "DSA prefill tokens/sec at T=64K, top-2048 (indexer+top-k+sparse MLA); % roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--T", type=int, default=65536, help="sequence length (default 65536)")
+    ap.add_argument("--topk", type=int, default=2048)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------------
+# workload
+# ----------------------------------------------------------------------------------
+def make_inputs(T, k, seed):
+    from sparse_attention_17_b200 import inputs as G
+    return G.mla_prefill_gauss(T=T, seed=seed, k=k)
+
+
+def algorithmic_work(T, k):
+    """FLOPs and bytes of one prefill step, counted from the definitions."""
+    causal = T * (T + 1) // 2                       # (t, s) pairs with s <= t
+    sel = sum(min(t + 1, k) for t in range(T))      # selected keys over all queries
+    return {
+        "indexer_flop": 2 * 16 * 64 * causal,       # 16 heads x 64-dim dot per pair
+        "mla_flop": 2 * 16 * (576 + 512) * sel,     # QK (576) + PV (512) per head per key
+        "mla_gather_bytes": 1152 * sel,             # one 576 x bf16 latent row per key
+        "topk_read_bytes": 4 * causal,              # fp32 scores read once per pair
+        "hbm_bytes": (T * 16 * 64 * 2 + T * 64 * 2 + T * 16 * 4 + T * 16 * 576 * 2
+                      + T * 576 * 2 + T * 16 * 512 * 2 + 2 * T * k * 4),
+    }
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(name):
+    h = hashlib.sha256()
+    for f in sorted((ROOT / "sparse_attention_17_b200" / "csrc").glob("*")):
+        if f.name in (name, "dsa_common.cuh"):
+            h.update(f.read_bytes())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel_file):
+    """DRAM traffic per launch from the committed ncu summary, if the kernel source has not
+    changed since it was taken."""
+    p = ROOT / "profiles" / "traffic.json"
+    if not p.exists():
+        return None
+    d = json.loads(p.read_text()).get(kernel_file)
+    if not d or d.get("source_hash") != kernel_source_hash(kernel_file):
+        return None
+    return d.get("bytes_per_launch_full")
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, _, r in rows:
+            for n, v in zip(names, r[1:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(x[0] for x in rows),
+                "sm_max_mhz": max(x[1] for x in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ----------------------------------------------------------------------------------
+def oracle_rows_throughput(d, k, seconds, rng_seed=0, max_rows=None):
+    """Runs the oracle's indexer + top-k + attention on blocks of consecutive query rows,
+    each block starting at a uniformly drawn position of the workload, until about
+    `seconds` of wall time are spent.  Each oracle call covers a whole block, so its
+    OpenMP loop spreads the rows over all host threads.  Returns (rows/s, rows, threads,
+    seconds)."""
+    import numpy as np
+    from oracle import oracle as O
+    T = d["q_idx"].shape[0]
+    r = np.random.default_rng(rng_seed)
+    q_idx, k_idx, w = (O._f32(d[n]) for n in ("q_idx", "k_idx", "w"))
+    q, kv = d["q"], O._f32(d["kv"])
+    threads = O.num_threads()
+    block = 2 * threads
+    done, t0 = 0, time.perf_counter()
+    while True:
+        b0 = int(r.integers(0, T - block + 1))
+        sc = O.indexer_scores_prefill(q_idx, k_idx, w, b0, block, b0 + block)
+        idx = O.topk(sc, O.causal_n_valid(b0, block), k)
+        O.sparse_mla_prefill(q[b0:b0 + block], kv, idx, 192 ** -0.5)
+        done += block
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_rows and done >= max_rows):
+            return done / el, done, threads, el
+
+
+# ----------------------------------------------------------------------------------
+# native arm
+# ----------------------------------------------------------------------------------
+def run_native(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import sparse_attention_17_b200 as dsa
+    from sparse_attention_17_b200 import inputs as G
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    T, k = args.T, args.topk
+    host = make_inputs(T, k, seed=rank)
+    names = ("q_idx", "k_idx", "w", "q", "kv")
+    x = {n: host[n].to(dev) for n in names}
+    ld = (T + 3) // 4 * 4
+    ws_bytes = dsa.layer_stack_workspace_size(T)
+    rw = max(16, ws_bytes // (4 * ld))
+    rw = min(T, rw // 16 * 16 if rw > 16 else rw)
+    scores = torch.empty((rw, ld), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    out = torch.empty((T, 16, 512), dtype=torch.bfloat16, device=dev)
+    windows = [(q0, min(rw, T - q0)) for q0 in range(0, T, rw)]
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        """One prefill pass through the public C ABI: indexer + top-k per window of query
+        rows into the index buffer, then sparse MLA over all queries."""
+        if ev is not None:
+            ev[0].record(stream)
+        for q0, rows in windows:
+            dsa.indexer_scores(x["q_idx"], x["k_idx"], x["w"], scores, q0, rows)
+            dsa.topk_select(scores, k, idx[q0:q0 + rows], q_begin=q0, rows=rows)
+        if ev is not None:
+            ev[1].record(stream)
+        dsa.sparse_mla_fwd(x["q"], x["kv"], idx, out, G.SCALE_MLA)
+        if ev is not None:
+            ev[2].record(stream)
+
+    def sync_all():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    assert dsa.check_device_errors() == 0
+    sync_all()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = [dsa.launch_count(i) for i in range(4)]
+    with ClockSampler(local_rank) as clk:
+        sync_all()
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    launches = sum(dsa.launch_count(i) - launches0[i] for i in range(4))
+    ms_total = start.elapsed_time(stop)
+    idx_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    mla_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    errs = dsa.check_device_errors()
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+
+    # per-kernel split of the index phase (separate, untimed-for-value pass)
+    e_idx = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(windows) + 1)]
+    torch.cuda.synchronize()
+    e_idx[0].record(stream)
+    for i, (q0, rows) in enumerate(windows):
+        dsa.indexer_scores(x["q_idx"], x["k_idx"], x["w"], scores, q0, rows)
+        e_idx[2 * i + 1].record(stream)
+        dsa.topk_select(scores, k, idx[q0:q0 + rows], q_begin=q0, rows=rows)
+        e_idx[2 * i + 2].record(stream)
+    torch.cuda.synchronize()
+    indexer_ms = sum(e_idx[2 * i].elapsed_time(e_idx[2 * i + 1]) for i in range(len(windows)))
+    topk_ms = sum(e_idx[2 * i + 1].elapsed_time(e_idx[2 * i + 2]) for i in range(len(windows)))
+
+    # end to end through the API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        pinned = {n: host[n].pin_memory() for n in names}
+        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+        d2h = out_host.numel() * out_host.element_size()
+
+        def e2e_step():
+            for n in names:
+                x[n].copy_(pinned[n], non_blocking=True)
+            step()
+            out_host.copy_(out, non_blocking=True)
+
+        e2e_step()
+        sync_all()
+        s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        n_e2e = max(1, min(args.steps, 5))
+        for _ in range(n_e2e):
+            e2e_step()
+        t2.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = s2.elapsed_time(t2) / n_e2e
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    result = None
+    if rank == 0:
+        work = algorithmic_work(T, k)
+        peaks, peak_src = load_peaks()
+        ms_step = ms_total / args.steps
+        value = world * T / (ms_step / 1e3)
+        kern = {"indexer_ms": indexer_ms, "topk_ms": topk_ms, "sparse_mla_ms": mla_ms,
+                "index_phase_ms": idx_ms}
+        # dominant kernel
+        if mla_ms >= indexer_ms:
+            dom, flop, fname = "sparse_mla_tc_kernel", work["mla_flop"], "mla_tc.cu"
+            dom_ms = mla_ms
+        else:
+            dom, flop, fname = "indexer_tc_kernel", work["indexer_flop"], "indexer_tc.cu"
+            dom_ms = indexer_ms
+        peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+        achieved = flop / (dom_ms / 1e3) / 1e12
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 2),
+                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "traffic": load_traffic(fname),
+                    "peak_source": f"{peak_src} bf16 dense, sustained (kernel timed inside a long step)"}
+        others = {
+            "indexer_tflops": round(work["indexer_flop"] / (indexer_ms / 1e3) / 1e12, 2),
+            "indexer_frac_of_burst_peak": round(work["indexer_flop"] / (indexer_ms / 1e3) / 1e12
+                                                / peaks.get("bf16_tflops", 1590.0), 4),
+            "sparse_mla_tflops": round(work["mla_flop"] / (mla_ms / 1e3) / 1e12, 2),
+            "sparse_mla_gather_gbs": round(work["mla_gather_bytes"] / (mla_ms / 1e3) / 1e9, 1),
+            "topk_score_read_gbs": round(work["topk_read_bytes"] / (topk_ms / 1e3) / 1e9, 1),
+            "step_roofline_ms": round((work["indexer_flop"] + work["mla_flop"]) / 1e12
+                                      / peak * 1e3, 3),
+        }
+        others["step_frac_of_roofline"] = round(others["step_roofline_ms"] / ms_step, 4)
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"dsa_prefill_T{T}_top{k}", "T": T, "topk": k,
+                       "batch_per_gpu": 1, "indexer_heads": 16, "indexer_dim": 64,
+                       "heads": 16, "latent_dim": 576, "value_dim": 512,
+                       "index_window_rows": rw, "parallelism": f"independent sequences x{world}",
+                       "l2": "inputs larger than L2 (%.2f GB per step), no flush" %
+                             (sum(t.numel() * t.element_size() for t in host.values()
+                                  if hasattr(t, "numel")) / 1e9)},
+            "roofline": roofline,
+            "kernels": {kk: round(v, 4) for kk, v in kern.items()},
+            "derived": others,
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+            "device_error_bits": errs,
+        }
+        if e2e is not None:
+            e2e["value"] = round(e2e["value"], 1)
+            e2e["ms_per_step"] = round(e2e["ms_per_step"], 3)
+            result["e2e"] = e2e
+        if not args.no_cpu_baseline and world == 1:
+            rps, n, cores, el = oracle_rows_throughput(host, k, args.cpu_seconds)
+            result["cpu_baseline"] = {
+                "value": round(rps, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"{n} query rows of the T={T} workload in blocks of "
+                          f"{2 * cores} consecutive rows at uniform positions (indexer + "
+                          f"top-k + attention, fp64), {el:.1f} s"}
+    return result
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle, as it stands, on bounded samples of the same workload."""
+    if rank != 0:
+        return None
+    T, k = args.T, args.topk
+    host = make_inputs(T, k, seed=0)
+    per_step = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_rows_throughput(host, k, per_step / 4, rng_seed=1)
+    vals, rows, secs = [], 0, 0.0
+    cores = 1
+    for i in range(args.steps):
+        rps, n, cores, el = oracle_rows_throughput(host, k, per_step, rng_seed=100 + i)
+        vals.append(rps)
+        rows += n
+        secs += el
+    value = rows / secs
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / value, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"dsa_prefill_T{T}_top{k}", "T": T, "topk": k},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{rows} query rows of the T={T} workload in blocks of "
+                                   f"{2 * cores} consecutive rows at uniform positions, "
+                                   f"{secs:.1f} s over {args.steps} steps"},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        res = run_native(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

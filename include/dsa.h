@@ -1,0 +1,222 @@
+/*
+ * dsa.h -- C ABI of the B200 (sm_100a) DeepSeek Sparse Attention hot path.
+ *
+ * The library computes, on one GPU, the three steps of DSA prefill and decode and the
+ * IndexCache reuse of selected indices across layers:
+ *
+ *   dsa_indexer_scores   lightning-indexer scores  I(t,s) = sum_j w[t,j] * ReLU(q_idx[t,j] . k_idx[s])
+ *   dsa_topk_select      per-row top-k of those scores (ties -> lower index), ascending, -1 padded
+ *   dsa_sparse_mla_fwd   attention of each query over its selected keys only (absorbed MLA:
+ *                        one 576-dim latent row per token shared by all heads, value = first
+ *                        512 dims; or plain multi-head attention for the fp32 path)
+ *   dsa_layer_stack      an F/S pattern of layers: F layers run indexer + top-k into one
+ *                        index buffer, S layers reuse it (IndexCache)
+ *
+ * Sources.  DSA ablation model card ("Attention" bullet: a ReLU lightning indexer picks the
+ * top-k keys per query; closing note: prompts no longer than k attend densely);
+ * DSV2-Lite-IndexCache-Sparse-1250 card (first paragraph: causal selection budget of 2048,
+ * FSS pattern repeated nine times, full layers' routes reused by shared layers);
+ * DeepSeek-V2-Lite-Chat SIQ card (MLA with kv_lora_rank 512, 576 B per token at fp8, i.e.
+ * a 576-element latent); vLLM IndexCache docs ("Configuration Reference": index_topk_freq
+ * and index_topk_pattern; "How It Works": F layers store top-k indices, S layers receive
+ * them).  The indexer formula itself is not printed on those pages; this library takes the
+ * standard DSA form above with one indexer key per token shared by all indexer heads.
+ *
+ * Conventions for every call:
+ *   - All tensor arguments are DEVICE pointers owned by the caller; the library never
+ *     allocates, frees or retains them.  Scratch memory is passed in as `workspace`.
+ *   - Tensors are dense row-major ("C order") unless a leading dimension is given.
+ *     Tensor pointers must be 16-byte aligned; leading dimensions are in elements.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream).  Results are valid once the stream has reached the call.
+ *   - Argument errors return DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED before anything is
+ *     launched; dsa_last_error() then describes the problem.  DSA_ERR_CUDA reports a
+ *     failed launch or CUDA runtime call.
+ *   - Indices handed to dsa_sparse_mla_fwd that fall outside the valid key range are
+ *     skipped by the kernel and recorded in a per-device error word, which
+ *     dsa_check_device_errors() reads and clears.  They never cause an out-of-bounds read.
+ *   - Results are deterministic: no floating-point atomics; identical inputs give
+ *     bit-identical outputs.
+ *   - Thread safety: calls may be issued from several host threads on different streams.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dsa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,  /* a pointer, size, stride or alignment is wrong */
+    DSA_ERR_UNSUPPORTED = 2,  /* a valid request this build has no kernel for */
+    DSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+    DSA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+    DSA_ERR_DEVICE_CHECK = 5  /* a kernel recorded an invalid input (see error bits) */
+} dsa_status;
+
+typedef enum { DSA_F32 = 0, DSA_BF16 = 1 } dsa_dtype;
+typedef enum { DSA_PREFILL = 0, DSA_DECODE = 1 } dsa_mode;
+
+/* Bits of the per-device error word (dsa_check_device_errors). */
+#define DSA_DEVERR_INDEX_RANGE 0x1u  /* a selected index outside [0, valid length) */
+#define DSA_DEVERR_PAGE_RANGE  0x2u  /* a page-table entry outside the page pool */
+#define DSA_DEVERR_TIMEOUT     0x4u  /* an internal pipeline wait gave up (kernel bug) */
+
+/* Kernel families counted by dsa_launch_count(). */
+typedef enum {
+    DSA_KERNEL_INDEXER = 0,
+    DSA_KERNEL_TOPK = 1,
+    DSA_KERNEL_ATTENTION = 2,
+    DSA_KERNEL_COMBINE = 3,
+    DSA_KERNEL_KINDS = 4
+} dsa_kernel_kind;
+
+/* Human-readable name of a status code (static storage). */
+const char* dsa_status_string(int status);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+const char* dsa_last_error(void);
+
+/* ABI version of this header: (major << 16) | minor. */
+int dsa_version(void);
+
+/*
+ * dsa_indexer_scores -- lightning indexer scores (DSA ablation card, "Attention" bullet).
+ *
+ *   I(t,s) = sum_{j < H_I} w[t,j] * max(0, sum_{d < D_I} q_idx[t,j,d] * k_idx[s,d])
+ *
+ * mode DSA_PREFILL (causal, DSV2-Lite-IndexCache card: causal key selection):
+ *   q_idx  [T, H_I, D_I]   dtype (bf16 or fp32), T >= q_begin + rows
+ *   k_idx  [S, D_I]        dtype, S >= q_begin + rows
+ *   w      [T, H_I]        fp32
+ *   Row r of `scores` is query t = q_begin + r; columns s = 0..t hold I(t,s).  Columns
+ *   t+1 .. ld_scores-1 are unspecified (the kernel may or may not write them).
+ *   page_table, seq_lens must be NULL; max_pages, page_size are ignored.
+ * mode DSA_DECODE (bf16 only; one new query per sequence, keys read through pages):
+ *   q_idx  [B, H_I, D_I]   with B = rows, q_begin = 0
+ *   k_idx  [num_pages, page_size, D_I] page pool; S = num_pages * page_size
+ *   w      [B, H_I]
+ *   page_table [B, max_pages] int32: token s of sequence b is pool row
+ *              page_table[b, s / page_size] * page_size + s % page_size
+ *   seq_lens   [B] int32: sequence b scores keys 0..seq_lens[b]-1 (the new token's key is
+ *              already in the cache); 1 <= seq_lens[b] <= min(ld_scores, max_pages*page_size).
+ *   Columns >= seq_lens[b] are unspecified.
+ * scores [rows, ld_scores] fp32, ld_scores a multiple of 4 and >= q_begin + rows (prefill).
+ * Supported: bf16 with H_I = 16, D_I = 64; fp32 (prefill only) with H_I * D_I <= 256 and
+ * D_I a multiple of 4.  Page sizes: multiples of 16 (decode).
+ */
+dsa_status dsa_indexer_scores(int dtype, int mode, const void* q_idx, const void* k_idx,
+                              const float* w, int H_I, int D_I, int q_begin, int rows, int S,
+                              const int* page_table, int max_pages, int page_size,
+                              const int* seq_lens, float* scores, long long ld_scores,
+                              dsa_stream_t stream);
+
+/*
+ * dsa_topk_select -- per-row top-k (DSA ablation card: top-k keys per query; its closing
+ * note: when a row has no more than k valid keys, all of them are selected).
+ *
+ * Row r has n_r valid scores in columns 0..n_r-1 of scores[r * ld_scores ...]:
+ *   row_len == NULL:  n_r = q_begin + r + 1          (causal prefill rows)
+ *   row_len != NULL:  n_r = row_len[r] (device int32) (decode rows)
+ * and 1 <= n_r <= max_len <= ld_scores.  Selection: the k valid keys with the largest
+ * scores; among equal scores the lower index wins (-0.0 and +0.0 are equal).  If n_r <= k
+ * all n_r keys are selected.  idx[r * ld_idx + i], i < k, receives the selected key
+ * positions in ascending order followed by -1 padding.  Scores must not be NaN.
+ * Limits: 1 <= k <= 4096, max_len <= 262144, ld_idx >= k.
+ */
+dsa_status dsa_topk_select(const float* scores, long long ld_scores, int rows, int q_begin,
+                           const int* row_len, int max_len, int k, int* idx,
+                           long long ld_idx, dsa_stream_t stream);
+
+/*
+ * dsa_sparse_mla_fwd -- attention over the selected keys only (DSV2-Lite-IndexCache card:
+ * attention_mode="sparse"; its portable runtime is the same computation as masked SDPA).
+ *
+ * For query n, head h, with I_n the non-negative entries of idx[n * ld_idx + 0 .. k_sel-1]:
+ *   logit_s = scale * q[n,h,:] . K(s)
+ *   out[n,h,:] = sum_{s in I_n} softmax_s(logit) * V(s)
+ *   lse[n,h]   = log sum_{s in I_n} exp(logit_s)            (natural log; -inf if I_n empty)
+ * MLA (dtype DSA_BF16, num_kv_heads = 1, v = NULL): K(s) is the latent row kv[s, 0:D_qk]
+ *   shared by all H heads and V(s) = kv[s, 0:D_v].  Supported: H = 16, D_qk = 576, D_v = 512.
+ * MHA (dtype DSA_F32, num_kv_heads = H, v != NULL): K(s) = kv[s,h,:], V(s) = v[s,h,:],
+ *   D_qk = D_v <= 64, H <= 16; prefill only.
+ *
+ * mode DSA_PREFILL:  q [num_q, H, D_qk]; kv [kv_rows, num_kv_heads, D_qk]; query n uses
+ *   the rows named by idx directly (0 <= s < kv_rows is checked).  page_table, seq_lens NULL.
+ * mode DSA_DECODE:   num_q = B sequences; kv is the page pool
+ *   [kv_rows / page_size pages, page_size, D_qk]; token s of sequence n lives in pool row
+ *   page_table[n, s / page_size] * page_size + s % page_size; only 0 <= s < seq_lens[n]
+ *   is valid.  The decode path splits each sequence's keys over several CTAs and merges
+ *   them with their log-sum-exp; it needs `workspace` of dsa_sparse_mla_workspace_size().
+ * out [num_q, H, D_v] in dtype; lse [num_q, H] fp32 or NULL.
+ * workspace may be NULL when dsa_sparse_mla_workspace_size() returns 0.
+ */
+dsa_status dsa_sparse_mla_fwd(int dtype, int mode, int num_q, int H, int num_kv_heads,
+                              int D_qk, int D_v, float scale, const void* q, const void* kv,
+                              const void* v, long long kv_rows, const int* page_table,
+                              int max_pages, int page_size, const int* seq_lens,
+                              const int* idx, int k_sel, long long ld_idx, void* out,
+                              float* lse, void* workspace, size_t workspace_bytes,
+                              dsa_stream_t stream);
+
+/* Workspace bytes dsa_sparse_mla_fwd needs for this shape (0 for prefill). */
+size_t dsa_sparse_mla_workspace_size(int mode, int num_q, int H, int D_v, int k_sel);
+
+/*
+ * dsa_layer_stack -- IndexCache over an F/S layer pattern (vLLM IndexCache docs, "How It
+ * Works"; DSV2-Lite-IndexCache card: "FSS" x 9).  Prefill, bf16 absorbed MLA.
+ *
+ * pattern: num_layers characters from {'F','S'}, pattern[0] == 'F'.
+ * For layer l (arrays are HOST arrays of DEVICE pointers, length num_layers):
+ *   'F': idx_buf <- top-k of the layer's own indexer scores
+ *        (q_idx[l] [T,16,64] bf16, k_idx[l] [T,64] bf16, w[l] [T,16] fp32), computed in
+ *        windows of query rows through `workspace`.
+ *   'S': idx_buf is reused unchanged (no indexer or top-k launch; q_idx[l], k_idx[l],
+ *        w[l] are not read and may be NULL).
+ *   every layer: out[l] [T,16,512] <- sparse MLA of q[l] [T,16,576] over kv[l] [T,576]
+ *        with the current idx_buf; lse[l] [T,16] fp32 if lse != NULL and lse[l] != NULL.
+ * idx_buf [T, topk] int32 holds, on return, the indices of the last F layer.
+ * workspace: at least dsa_layer_stack_workspace_size(T, 0) bytes; a larger workspace
+ * processes more query rows per window.
+ */
+dsa_status dsa_layer_stack(const char* pattern, int num_layers, int T, int topk,
+                           int H_I, int D_I, int H, int D_qk, int D_v, float scale,
+                           const void* const* q_idx, const void* const* k_idx,
+                           const float* const* w, const void* const* q,
+                           const void* const* kv, void* const* out, float* const* lse,
+                           int* idx_buf, void* workspace, size_t workspace_bytes,
+                           dsa_stream_t stream);
+
+/* Workspace bytes for dsa_layer_stack with windows of rows_window query rows
+ * (0 = the library's default window). */
+size_t dsa_layer_stack_workspace_size(int T, int rows_window);
+
+/*
+ * dsa_pattern_from_freq -- the pattern index_topk_freq describes (vLLM IndexCache docs,
+ * "Configuration Reference": top-k computed every freq layers; freq 1 = every layer).
+ * Layer i is 'F' iff i % freq == 0.  Writes num_layers characters and a NUL into
+ * out[0 .. out_len-1]; out_len must be > num_layers.  Host-only.
+ */
+dsa_status dsa_pattern_from_freq(int freq, int num_layers, char* out, int out_len);
+
+/* Reads and clears the current device's error word after synchronizing `stream`.
+ * *error_bits (may be NULL) receives the DSA_DEVERR_* bits.  Returns
+ * DSA_ERR_DEVICE_CHECK if any bit was set, DSA_OK otherwise. */
+dsa_status dsa_check_device_errors(dsa_stream_t stream, unsigned* error_bits);
+
+/* Number of kernels of a family this process has launched through the library (all
+ * devices, all threads); used to check that S layers launch no indexer or top-k. */
+long long dsa_launch_count(int kind);
+void dsa_reset_launch_counts(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

@@ -1,0 +1,360 @@
+// indexer_tc.cu -- lightning-indexer scores on tcgen05 tensor cores (bf16 in, fp32 out).
+//
+//   I(t,s) = sum_{j<16} w[t,j] * max(0, sum_{d<64} q_idx[t,j,d] * k_idx[s,d])
+//
+// (DSA ablation card, "Attention" bullet: a ReLU lightning indexer scores every key per
+// query; one indexer key per token is shared by the heads.)
+//
+// Tiling.  Keys go on the UMMA M side (128 keys = the 128 TMEM lanes) and (query, head)
+// pairs on the N side: N = QB * 16 with QB = 16 queries per block in prefill and QB = 1 in
+// decode.  K = 64 is a single 128-byte swizzle atom, so one tile is 4 UMMAs of K = 16.
+// With keys on lanes, the ReLU + head-weight reduction of a score is a sum over 16
+// consecutive TMEM columns that stay inside one thread -- no shuffles.
+//
+// Warp roles (384 threads): warp 0 issues TMA loads (query block once per unit, key tiles
+// through a ring of smem stages), warp 1 issues UMMAs into a double-buffered TMEM
+// accumulator (2 x 256 columns), warp 2 owns the TMEM allocation, warps 4..11 drain the
+// accumulator: tcgen05.ld, ReLU, weight, reduce, causal mask, coalesced fp32 stores.
+//
+// Prefill units are blocks of 16 queries; their causal key range grows with the query
+// position, so persistent CTAs take units in snake order to even out the triangle.
+// Decode units are (sequence, 2048-key chunk); key tiles are assembled from pages with one
+// TMA load per page.
+#include "dsa_common.cuh"
+#include "launch.h"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kHI = 16;
+constexpr int kDI = 64;
+constexpr int kBM = 128;           // keys per tile (UMMA M)
+constexpr int kStages = 6;         // key-tile ring
+constexpr int kThreads = 384;
+constexpr int kEpiWarp0 = 4;       // first epilogue warp
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kTileBytes = kBM * 128;  // 128 keys x 64 bf16
+constexpr int kDecodeChunkTiles = 16;       // decode unit = 2048 keys
+
+template <int QB>
+struct IdxSmem {
+    alignas(1024) uint8_t k[kStages][kTileBytes];
+    alignas(1024) uint8_t q[QB * kHI * 128 < 1024 ? 1024 : QB * kHI * 128];
+    float w[kEpiWarps][QB >= 2 ? QB / 2 * kHI : kHI];  // per-warp head weights of its queries
+    uint64_t k_full[kStages];
+    uint64_t k_empty[kStages];
+    uint64_t q_full, q_empty;
+    uint64_t acc_full[2], acc_empty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct IdxParams {
+    const float* w;
+    float* scores;
+    long long ld;
+    int q_begin, q_end;  // prefill query rows [q_begin, q_end)
+    int S;               // prefill: key rows
+    int num_units;
+    // decode
+    const int* page_table;
+    const int* seq_lens;
+    int max_pages, page_size, num_pages, max_len;
+    unsigned* err;
+};
+
+// Unit visited by this CTA at step i (snake order over rounds of gridDim.x units).
+__device__ __forceinline__ int unit_at(int i) {
+    const int G = gridDim.x, c = blockIdx.x;
+    return (i & 1) ? i * G + (G - 1 - c) : i * G + c;
+}
+
+template <int QB, bool PAGED>
+struct UnitInfo {
+    int row0;       // prefill: first query t0; decode: sequence b
+    int tile0;      // first key tile
+    int ntiles;     // key tiles in this unit
+    int len;        // decode: valid keys of the sequence
+};
+
+template <int QB, bool PAGED>
+__device__ __forceinline__ UnitInfo<QB, PAGED> unit_info(const IdxParams& p, int u) {
+    UnitInfo<QB, PAGED> x;
+    if constexpr (!PAGED) {
+        x.row0 = p.q_begin + u * QB;
+        const int t_max = min(x.row0 + QB, p.q_end) - 1;
+        x.tile0 = 0;
+        x.ntiles = t_max / kBM + 1;
+        x.len = 0;
+    } else {
+        const int units_per_seq = (p.max_len + kBM * kDecodeChunkTiles - 1) / (kBM * kDecodeChunkTiles);
+        x.row0 = u / units_per_seq;
+        const int chunk = u % units_per_seq;
+        int len = __ldg(p.seq_lens + x.row0);
+        len = max(0, min(len, p.max_len));
+        x.len = len;
+        x.tile0 = chunk * kDecodeChunkTiles;
+        const int tiles_total = (len + kBM - 1) / kBM;
+        x.ntiles = max(0, min(kDecodeChunkTiles, tiles_total - x.tile0));
+    }
+    return x;
+}
+
+template <int QB, bool PAGED>
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                  const __grid_constant__ CUtensorMap tmap_k, const IdxParams p) {
+    constexpr int BN = QB * kHI;                     // UMMA N
+    constexpr uint32_t kQBytes = BN * 128;
+    constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;  // TMEM columns per accumulator
+    constexpr uint32_t kTmemCols = 2 * kAccCols <= 32 ? 32 : (2 * kAccCols <= 64 ? 64 : (2 * kAccCols <= 128 ? 128 : (2 * kAccCols <= 256 ? 256 : 512)));
+    constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, 0, 0);
+    using Smem = IdxSmem<QB>;
+
+    extern __shared__ uint8_t smem_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    volatile int* abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&sm.k_full[i], 1);
+            mbar_init(&sm.k_empty[i], 1);
+        }
+        mbar_init(&sm.q_full, 1);
+        mbar_init(&sm.q_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.acc_full[i], 1);
+            mbar_init(&sm.acc_empty[i], kEpiWarps);
+        }
+        sm.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------- TMA producer ----------------
+        tma_prefetch_desc(&tmap_q);
+        tma_prefetch_desc(&tmap_k);
+        uint32_t it = 0;
+        for (int i = 0, ui = 0;; ++i, ++ui) {
+            const int u = unit_at(i);
+            if (u >= p.num_units) break;
+            const UnitInfo<QB, PAGED> x = unit_info<QB, PAGED>(p, u);
+            if (!mbar_wait(&sm.q_empty, (ui & 1) ^ 1, abort, p.err)) break;
+            mbar_arrive_expect_tx(&sm.q_full, kQBytes);
+            tma_load_2d(sm.q, &tmap_q, 0, x.row0 * kHI, &sm.q_full);
+            bool ok = true;
+            for (int j = 0; j < x.ntiles; ++j, ++it) {
+                const int st = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                if (!mbar_wait(&sm.k_empty[st], ph ^ 1, abort, p.err)) { ok = false; break; }
+                const int tile = x.tile0 + j;
+                if constexpr (!PAGED) {
+                    mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
+                    tma_load_2d(sm.k[st], &tmap_k, 0, tile * kBM, &sm.k_full[st]);
+                } else {
+                    const int ps = p.page_size;
+                    const int per = kBM / ps;
+                    const int page0 = tile * per;
+                    const int used = min(per, (x.len - tile * kBM + ps - 1) / ps);
+                    mbar_arrive_expect_tx(&sm.k_full[st], (uint32_t)(used * ps * 128));
+                    for (int q = 0; q < used; ++q) {
+                        int pg = __ldg(p.page_table + (long long)x.row0 * p.max_pages + page0 + q);
+                        if (pg < 0 || pg >= p.num_pages) {
+                            atomicOr(p.err, DSA_DEVERR_PAGE_RANGE);
+                            pg = 0;
+                        }
+                        tma_load_2d(sm.k[st] + q * ps * 128, &tmap_k, 0, pg * ps, &sm.k_full[st]);
+                    }
+                }
+            }
+            if (!ok) break;
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---------------- UMMA issuer ----------------
+        const uint32_t q_addr = smem_u32(sm.q);
+        uint32_t it = 0;
+        for (int i = 0, ui = 0;; ++i, ++ui) {
+            const int u = unit_at(i);
+            if (u >= p.num_units) break;
+            const UnitInfo<QB, PAGED> x = unit_info<QB, PAGED>(p, u);
+            if (!mbar_wait(&sm.q_full, ui & 1, abort, p.err)) break;
+            bool ok = true;
+            for (int j = 0; j < x.ntiles; ++j, ++it) {
+                const int st = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                const int ab = it & 1;
+                const uint32_t aph = (it >> 1) & 1;
+                if (!mbar_wait(&sm.k_full[st], ph, abort, p.err)) { ok = false; break; }
+                if (!mbar_wait(&sm.acc_empty[ab], aph ^ 1, abort, p.err)) { ok = false; break; }
+                tc_fence_after();
+                const uint64_t adesc = smem_desc(smem_u32(sm.k[st]), 16, 1024, kSwizzle128B);
+                const uint64_t bdesc = smem_desc(q_addr, 16, 1024, kSwizzle128B);
+#pragma unroll
+                for (int kk = 0; kk < kDI / 16; ++kk)
+                    umma_bf16(tmem + ab * kAccCols, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, kk > 0);
+                umma_commit(&sm.k_empty[st]);
+                umma_commit(&sm.acc_full[ab]);
+            }
+            umma_commit(&sm.q_empty);
+            if (!ok) break;
+        }
+    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiWarps) {
+        // ---------------- epilogue ----------------
+        const int ew = warp - kEpiWarp0;
+        const int quad = warp & 3;              // TMEM lane quadrant this warp may access
+        const int half = ew >> 2;               // which half of the queries
+        constexpr int QPW = QB >= 2 ? QB / 2 : 1;  // queries per epilogue warp
+        const bool active_half = QB >= 2 || half == 0;
+        uint32_t it = 0;
+        for (int i = 0, ui = 0;; ++i, ++ui) {
+            const int u = unit_at(i);
+            if (u >= p.num_units) break;
+            const UnitInfo<QB, PAGED> x = unit_info<QB, PAGED>(p, u);
+            // this warp's queries' head weights (warp-private; no cross-warp barrier)
+            float* wbuf = sm.w[ew];
+            __syncwarp();
+            for (int e = lane; e < QPW * kHI; e += 32) {
+                const int qidx = half * QPW + e / kHI;
+                const int t = x.row0 + qidx;
+                const bool valid = active_half && (PAGED ? true : (t < p.q_end));
+                wbuf[e] = valid ? __ldg(p.w + (long long)t * kHI + (e % kHI)) : 0.f;
+            }
+            __syncwarp();
+            bool ok = true;
+            for (int j = 0; j < x.ntiles; ++j, ++it) {
+                const int ab = it & 1;
+                const uint32_t aph = (it >> 1) & 1;
+                if (!mbar_wait(&sm.acc_full[ab], aph, abort, p.err)) { ok = false; break; }
+                tc_fence_after();
+                const int s = (x.tile0 + j) * kBM + quad * 32 + lane;
+                const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + ab * kAccCols;
+                if (active_half) {
+#pragma unroll
+                    for (int qi = 0; qi < QPW; qi += 2) {
+                        uint32_t ra[16], rb[16];
+                        const int i0 = half * QPW + qi;
+                        tmem_ld16(tbase + i0 * kHI, ra);
+                        if (QPW > 1) tmem_ld16(tbase + (i0 + 1) * kHI, rb);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int h2 = 0; h2 < (QPW > 1 ? 2 : 1); ++h2) {
+                            const int qidx = i0 + h2;
+                            const uint32_t* r = h2 == 0 ? ra : rb;
+                            const float4* w4 = reinterpret_cast<const float4*>(wbuf + (qidx - half * QPW) * kHI);
+                            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                            for (int h4 = 0; h4 < 4; ++h4) {
+                                const float4 wv = w4[h4];
+                                acc0 = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * h4 + 0]), 0.f), acc0);
+                                acc1 = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * h4 + 1]), 0.f), acc1);
+                                acc0 = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * h4 + 2]), 0.f), acc0);
+                                acc1 = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * h4 + 3]), 0.f), acc1);
+                            }
+                            const float score = acc0 + acc1;
+                            if constexpr (!PAGED) {
+                                const int t = x.row0 + qidx;
+                                if (t < p.q_end && s <= t)
+                                    p.scores[(long long)(t - p.q_begin) * p.ld + s] = score;
+                            } else {
+                                if (s < x.len) p.scores[(long long)x.row0 * p.ld + s] = score;
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
+            }
+            if (!ok) break;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int QB, bool PAGED>
+size_t indexer_smem_bytes() {
+    return sizeof(IdxSmem<QB>) + 1024;
+}
+
+template <int QB, bool PAGED>
+cudaError_t launch_indexer_tc(const CUtensorMap& tq, const CUtensorMap& tk, const IdxParams& p,
+                              int grid, cudaStream_t stream) {
+    const size_t smem = indexer_smem_bytes<QB, PAGED>();
+    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<QB, PAGED>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    indexer_tc_kernel<QB, PAGED><<<grid, kThreads, smem, stream>>>(tq, tk, p);
+    count_launch(DSA_KERNEL_INDEXER);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_indexer_bf16_prefill(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_idx,
+                                        const float* w, int T, int S, int q_begin, int rows,
+                                        float* scores, long long ld, cudaStream_t stream,
+                                        const DevCtx& ctx) {
+    constexpr int QB = 16;
+    CUtensorMap tq, tk;
+    if (!make_tmap_bf16_2d(&tq, q_idx, (uint64_t)T * kHI, kDI, kDI * 2, QB * kHI, kDI))
+        return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tk, k_idx, (uint64_t)S, kDI, kDI * 2, kBM, kDI))
+        return cudaErrorInvalidValue;
+    IdxParams p{};
+    p.w = w;
+    p.scores = scores;
+    p.ld = ld;
+    p.q_begin = q_begin;
+    p.q_end = q_begin + rows;
+    p.S = S;
+    p.num_units = (rows + QB - 1) / QB;
+    p.err = ctx.err;
+    const int grid = p.num_units < ctx.num_sms ? p.num_units : ctx.num_sms;
+    return launch_indexer_tc<QB, false>(tq, tk, p, grid, stream);
+}
+
+cudaError_t launch_indexer_bf16_decode(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_pool,
+                                       const float* w, int B, long long pool_rows,
+                                       const int* page_table, int max_pages, int page_size,
+                                       const int* seq_lens, int max_len, float* scores,
+                                       long long ld, cudaStream_t stream, const DevCtx& ctx) {
+    CUtensorMap tq, tk;
+    if (!make_tmap_bf16_2d(&tq, q_idx, (uint64_t)B * kHI, kDI, kDI * 2, kHI, kDI))
+        return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tk, k_pool, (uint64_t)pool_rows, kDI, kDI * 2, page_size, kDI))
+        return cudaErrorInvalidValue;
+    IdxParams p{};
+    p.w = w;
+    p.scores = scores;
+    p.ld = ld;
+    p.page_table = page_table;
+    p.seq_lens = seq_lens;
+    p.max_pages = max_pages;
+    p.page_size = page_size;
+    p.num_pages = (int)(pool_rows / page_size);
+    p.max_len = max_len;
+    const int units_per_seq = (max_len + kBM * kDecodeChunkTiles - 1) / (kBM * kDecodeChunkTiles);
+    p.num_units = B * units_per_seq;
+    p.err = ctx.err;
+    const int grid = p.num_units < ctx.num_sms ? p.num_units : ctx.num_sms;
+    return launch_indexer_tc<1, true>(tq, tk, p, grid, stream);
+}
+
+}  // namespace dsa

@@ -1,0 +1,325 @@
+// topk.cu -- per-row top-k of fp32 indexer scores by radix selection (no sort).
+//
+// Selection rule (DSA ablation card, "Attention" bullet and closing note): the k largest
+// of the row's n valid scores, equal scores resolved towards the lower key index; if
+// n <= k every key is selected.  Output: the selected key positions in ascending order,
+// then -1 padding.
+//
+// One CTA of 512 threads per row.  Scores map to order-preserving uint32 keys and the
+// k-th largest key (tau) is found one radix digit at a time (12 + 12 + 8 bits):
+//   pass 1  (global read)  histogram of bits 31..20 -> digit b1 holding the k-th key;
+//   pass 2  (global read)  keys with digit > b1 are selected (a bitmap word per warp
+//           ballot); keys with digit == b1 are appended to a candidate list in shared
+//           memory;
+//   refine  (shared memory) two more digit histograms over the candidates give tau;
+//           candidates above tau are selected, those equal to tau marked as ties.
+// If the b1 bucket is larger than the candidate buffer, the refinement reads the row
+// from global memory again instead (correct for any input, e.g. all scores equal).
+// Finally the first `need` ties in index order are kept and the bitmap is compacted in
+// index order, which yields ascending indices without sorting.
+#include "dsa_common.cuh"
+#include "launch.h"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBins = 4096;
+constexpr int kCandCap = 8192;
+constexpr int kStride = kWarps * 32;  // elements covered by all warps per iteration
+
+struct TopkScratch {
+    uint32_t hist[kBins];
+    uint32_t cand_key[kCandCap];
+    int cand_idx[kCandCap];
+    uint32_t scan[kWarps];
+    uint32_t cand_count;
+    uint32_t found_bin;
+    uint32_t found_above;
+};
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Adds 1 to hist[bin] for every lane with pred, one shared atomic per distinct bin.
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool pred) {
+    const unsigned active = __ballot_sync(0xffffffffu, pred);
+    if (pred) {
+        const unsigned peers = __match_any_sync(active, bin);
+        if ((int)lane_id() == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+    }
+}
+
+// Exclusive prefix sum over the block's threads (in thread order); *total gets the sum.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, TopkScratch& sh,
+                                                         uint32_t* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) sh.scan[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t w = lane < kWarps ? sh.scan[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < kWarps) sh.scan[lane] = w;
+    }
+    __syncthreads();
+    const uint32_t before = (warp > 0 ? sh.scan[warp - 1] : 0u) + x - v;
+    *total = sh.scan[kWarps - 1];
+    __syncthreads();
+    return before;
+}
+
+// Finds the bin b (scanning from the top) with above(b) < need <= above(b) + hist[b],
+// above(b) = number of keys in bins higher than b.  Result in sh.found_bin/found_above.
+__device__ void find_bin(TopkScratch& sh, int nbins, uint32_t need) {
+    const int per = nbins >= kThreads ? nbins / kThreads : 1;
+    const int first = nbins - 1 - (int)threadIdx.x * per;  // this thread's highest bin
+    uint32_t local = 0;
+    if (first >= 0)
+        for (int i = 0; i < per; ++i) local += sh.hist[first - i];
+    uint32_t total;
+    uint32_t above = block_exclusive_scan(local, sh, &total);
+    if (first >= 0 && above < need && above + local >= need) {
+        for (int i = 0; i < per; ++i) {
+            const uint32_t c = sh.hist[first - i];
+            if (above + c >= need) {
+                sh.found_bin = (uint32_t)(first - i);
+                sh.found_above = above;
+                break;
+            }
+            above += c;
+        }
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ void zero_hist(TopkScratch& sh, int nbins) {
+    for (int i = threadIdx.x; i < nbins; i += kThreads) sh.hist[i] = 0u;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
+                  const int* __restrict__ row_len, int max_len, int k, int* __restrict__ idx,
+                  long long ld_idx, unsigned* __restrict__ err) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    TopkScratch& sh = *reinterpret_cast<TopkScratch*>(smem_raw);
+    uint32_t* sel = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkScratch));
+    const int max_words = (max_len + 31) >> 5;
+    uint32_t* tie = sel + max_words;
+
+    const int r = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int n;
+    if (row_len != nullptr) {
+        n = row_len[r];
+        if (n < 0 || n > max_len) {
+            if (threadIdx.x == 0) atomicOr(err, DSA_DEVERR_INDEX_RANGE);
+            n = n < 0 ? 0 : max_len;
+        }
+    } else {
+        n = q_begin + r + 1;
+    }
+    int* out = idx + (long long)r * ld_idx;
+    if (n <= k) {  // every valid key is selected
+        for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    const float* row = scores + (long long)r * ld;
+    const int nwords = (n + 31) >> 5;
+
+    // ---- pass 1: histogram of the top 12 key bits over the whole row ----
+    zero_hist(sh, kBins);
+    for (int i = threadIdx.x; i < nwords; i += kThreads) tie[i] = 0u;
+    if (threadIdx.x == 0) sh.cand_count = 0u;
+    __syncthreads();
+    for (int base = warp * 32; base < n; base += 4 * kStride) {
+        float x[4];
+        bool in[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int s = base + u * kStride + lane;
+            in[u] = s < n;
+            x[u] = in[u] ? __ldg(row + s) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) hist_add(sh.hist, float_order_key(x[u]) >> 20, in[u]);
+    }
+    __syncthreads();
+    find_bin(sh, kBins, (uint32_t)k);
+    const uint32_t b1 = sh.found_bin;
+    uint32_t need = (uint32_t)k - sh.found_above;
+    const uint32_t cnt1 = sh.hist[b1];
+    __syncthreads();
+
+    uint32_t tau;
+    if (cnt1 <= (uint32_t)kCandCap) {
+        // ---- pass 2: definite selections to the bitmap, the b1 bucket to shared memory ----
+        for (int base = warp * 32; base < n; base += kStride) {
+            const int s = base + lane;
+            const bool in = s < n;
+            const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
+            const uint32_t hi = key >> 20;
+            const unsigned gt = __ballot_sync(0xffffffffu, in && hi > b1);
+            const bool eq = in && hi == b1;
+            const unsigned meq = __ballot_sync(0xffffffffu, eq);
+            if (lane == 0) sel[base >> 5] = gt;
+            if (meq) {
+                uint32_t pos0 = 0;
+                if (lane == 0) pos0 = atomicAdd(&sh.cand_count, (uint32_t)__popc(meq));
+                pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+                if (eq) {
+                    const uint32_t p = pos0 + __popc(meq & lanemask_lt());
+                    sh.cand_key[p] = key;
+                    sh.cand_idx[p] = s;
+                }
+            }
+        }
+        zero_hist(sh, kBins);
+        __syncthreads();
+        const int cnt = (int)sh.cand_count;
+        // ---- refine: bits 19..8 ----
+        for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
+            const int c = c0 + lane;
+            const bool in = c < cnt;
+            hist_add(sh.hist, in ? (sh.cand_key[c] >> 8) & 0xFFFu : 0u, in);
+        }
+        __syncthreads();
+        find_bin(sh, kBins, need);
+        const uint32_t b2 = sh.found_bin;
+        need -= sh.found_above;
+        zero_hist(sh, 256);
+        __syncthreads();
+        // ---- refine: bits 7..0 ----
+        const uint32_t pre = (b1 << 12) | b2;
+        for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
+            const int c = c0 + lane;
+            const uint32_t key = c < cnt ? sh.cand_key[c] : 0u;
+            const bool in = c < cnt && (key >> 8) == pre;
+            hist_add(sh.hist, key & 0xFFu, in);
+        }
+        __syncthreads();
+        find_bin(sh, 256, need);
+        need -= sh.found_above;
+        tau = (pre << 8) | sh.found_bin;
+        for (int c = threadIdx.x; c < cnt; c += kThreads) {
+            const uint32_t key = sh.cand_key[c];
+            const int s = sh.cand_idx[c];
+            if (key > tau) atomicOr(&sel[s >> 5], 1u << (s & 31));
+            else if (key == tau) atomicOr(&tie[s >> 5], 1u << (s & 31));
+        }
+    } else {
+        // ---- the b1 bucket does not fit: refine from global memory ----
+        zero_hist(sh, kBins);
+        __syncthreads();
+        for (int base = warp * 32; base < n; base += kStride) {
+            const int s = base + lane;
+            const bool in = s < n;
+            const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
+            hist_add(sh.hist, (key >> 8) & 0xFFFu, in && (key >> 20) == b1);
+        }
+        __syncthreads();
+        find_bin(sh, kBins, need);
+        const uint32_t b2 = sh.found_bin;
+        need -= sh.found_above;
+        zero_hist(sh, 256);
+        __syncthreads();
+        const uint32_t pre = (b1 << 12) | b2;
+        for (int base = warp * 32; base < n; base += kStride) {
+            const int s = base + lane;
+            const bool in = s < n;
+            const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
+            hist_add(sh.hist, key & 0xFFu, in && (key >> 8) == pre);
+        }
+        __syncthreads();
+        find_bin(sh, 256, need);
+        need -= sh.found_above;
+        tau = (pre << 8) | sh.found_bin;
+        for (int base = warp * 32; base < n; base += kStride) {
+            const int s = base + lane;
+            const bool in = s < n;
+            const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
+            const unsigned gt = __ballot_sync(0xffffffffu, in && key > tau);
+            const unsigned eq = __ballot_sync(0xffffffffu, in && key == tau);
+            if (lane == 0) {
+                sel[base >> 5] = gt;
+                tie[base >> 5] = eq;
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- keep the first `need` ties in index order, merge, compact ascending ----
+    const int wpt = (nwords + kThreads - 1) / kThreads;
+    const int w0 = threadIdx.x * wpt;
+    const int w1 = min(w0 + wpt, nwords);
+    uint32_t local = 0;
+    for (int w = w0; w < w1; ++w) local += __popc(tie[w]);
+    uint32_t total;
+    uint32_t before = block_exclusive_scan(local, sh, &total);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t tb = tie[w];
+        const uint32_t c = __popc(tb);
+        if (before >= need) {
+            tb = 0u;
+        } else if (before + c > need) {
+            uint32_t keep = 0u, rest = tb;
+            for (uint32_t m = need - before; m > 0; --m) {
+                keep |= rest & (0u - rest);
+                rest &= rest - 1u;
+            }
+            tb = keep;
+        }
+        before += c;
+        sel[w] |= tb;
+    }
+    __syncthreads();
+    local = 0;
+    for (int w = w0; w < w1; ++w) local += __popc(sel[w]);
+    uint32_t pos = block_exclusive_scan(local, sh, &total);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t bits = sel[w];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1u;
+            if (pos < (uint32_t)k) out[pos] = w * 32 + b;
+            ++pos;
+        }
+    }
+    for (int i = (int)total + threadIdx.x; i < k; i += kThreads) out[i] = -1;
+}
+
+}  // namespace
+
+size_t topk_smem_bytes(int max_len) {
+    const size_t words = (size_t)(max_len + 31) / 32;
+    return sizeof(TopkScratch) + 2 * words * sizeof(uint32_t);
+}
+
+cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin,
+                        const int* row_len, int max_len, int k, int* idx, long long ld_idx,
+                        cudaStream_t stream, const DevCtx& ctx) {
+    const size_t smem = topk_smem_bytes(max_len);
+    cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topk_radix_kernel<<<rows, kThreads, smem, stream>>>(scores, ld, q_begin, row_len, max_len, k,
+                                                        idx, ld_idx, ctx.err);
+    count_launch(DSA_KERNEL_TOPK);
+    return cudaGetLastError();
+}
+
+}  // namespace dsa

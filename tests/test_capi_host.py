@@ -1,0 +1,144 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol
+include/dsa.h declares, and rejects bad arguments before launching anything."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import sparse_attention_17_b200 as dsa
+from sparse_attention_17_b200 import _lib
+from oracle import oracle as O
+
+HEADER = Path(__file__).resolve().parents[1] / "include" / "dsa.h"
+
+
+def _declared():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return dsa.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), f"libdsa.so does not export {n}"
+    bound = {n for n, _, _ in _lib.SYMBOLS}
+    assert set(names) <= bound, set(names) - bound
+
+
+def test_version_and_status_strings(lib):
+    assert lib.dsa_version() >> 16 == 1
+    for code, name in enumerate(["DSA_OK", "DSA_ERR_INVALID_ARG", "DSA_ERR_UNSUPPORTED",
+                                 "DSA_ERR_WORKSPACE", "DSA_ERR_CUDA", "DSA_ERR_DEVICE_CHECK"]):
+        assert lib.dsa_status_string(code).decode() == name
+    assert lib.dsa_status_string(99).decode() == "DSA_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("freq,n", [(1, 5), (2, 7), (3, 27), (4, 61), (100, 3)])
+def test_pattern_from_freq_matches_oracle_reading(freq, n):
+    assert dsa.pattern_from_freq(freq, n) == O.pattern_from_freq(freq, n)
+
+
+def test_pattern_from_freq_rejects(lib):
+    buf = ctypes.create_string_buffer(4)
+    assert lib.dsa_pattern_from_freq(0, 3, buf, 4) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_pattern_from_freq(2, 4, buf, 4) == _lib.DSA_ERR_INVALID_ARG  # no room for NUL
+
+
+def _arr(n, v=16):
+    return (ctypes.c_void_p * n)(*([v] * n))
+
+
+@pytest.mark.parametrize("pattern,n,msg", [
+    (b"SFF", 3, "start"),
+    (b"FXS", 3, "not F or S"),
+    (b"FS", 3, "length"),
+    (b"", 0, "empty"),
+])
+def test_layer_stack_rejects_bad_patterns(lib, pattern, n, msg):
+    a = _arr(max(n, 1))
+    st = lib.dsa_layer_stack(pattern, n, 128, 64, 16, 64, 16, 576, 512, 0.1, a, a, a, a, a, a,
+                             None, 16, 16, 1 << 20, None)
+    assert st == _lib.DSA_ERR_INVALID_ARG
+    assert msg in lib.dsa_last_error().decode()
+
+
+def test_layer_stack_rejects_missing_indexer_inputs_of_f_layer(lib):
+    a = _arr(3)
+    none = (ctypes.c_void_p * 3)(16, 16, None)
+    st = lib.dsa_layer_stack(b"FSF", 3, 128, 64, 16, 64, 16, 576, 512, 0.1, none, a, a, a, a, a,
+                             None, 16, 16, 1 << 20, None)
+    assert st == _lib.DSA_ERR_INVALID_ARG and "F layer 2" in lib.dsa_last_error().decode()
+    # S layers may pass NULL indexer inputs: this one fails later, on the workspace
+    none_s = (ctypes.c_void_p * 3)(16, None, None)
+    st = lib.dsa_layer_stack(b"FSS", 3, 128, 64, 16, 64, 16, 576, 512, 0.1, none_s, none_s,
+                             none_s, a, a, a, None, 16, 16, 64, None)
+    assert st == _lib.DSA_ERR_WORKSPACE
+
+
+def test_layer_stack_rejects_unsupported_shapes(lib):
+    a = _arr(1)
+    st = lib.dsa_layer_stack(b"F", 1, 128, 64, 2, 16, 4, 32, 32, 0.1, a, a, a, a, a, a, None,
+                             16, 16, 1 << 20, None)
+    assert st == _lib.DSA_ERR_UNSUPPORTED
+
+
+def test_indexer_rejects_null_and_misaligned(lib):
+    st = lib.dsa_indexer_scores(1, 0, None, 16, 16, 16, 64, 0, 8, 8, None, 0, 0, None, 16, 8, None)
+    assert st == _lib.DSA_ERR_INVALID_ARG
+    st = lib.dsa_indexer_scores(1, 0, 18, 16, 16, 16, 64, 0, 8, 8, None, 0, 0, None, 16, 8, None)
+    assert st == _lib.DSA_ERR_INVALID_ARG and "aligned" in lib.dsa_last_error().decode()
+    st = lib.dsa_indexer_scores(1, 0, 16, 16, 16, 16, 64, 0, 8, 8, None, 0, 0, None, 16, 6, None)
+    assert st == _lib.DSA_ERR_INVALID_ARG and "multiple of 4" in lib.dsa_last_error().decode()
+    # zero rows is a valid no-op and touches no device
+    assert lib.dsa_indexer_scores(1, 0, 16, 16, 16, 16, 64, 0, 0, 8, None, 0, 0, None, 16, 8,
+                                  None) == _lib.DSA_OK
+
+
+def test_topk_rejects(lib):
+    assert lib.dsa_topk_select(16, 64, 4, 0, None, 64, 0, 16, 4, None) == _lib.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_topk_select(16, 64, 4, 0, None, 64, 5000, 16, 5000, None) == _lib.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_topk_select(16, 64, 4, 0, None, 64, 8, 16, 4, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk_select(16, 32, 4, 0, None, 64, 8, 16, 8, None) == _lib.DSA_ERR_INVALID_ARG
+    # causal rows beyond max_len
+    assert lib.dsa_topk_select(16, 64, 70, 0, None, 64, 8, 16, 8, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk_select(16, 64, 0, 0, None, 64, 8, 16, 8, None) == _lib.DSA_OK
+
+
+def test_attention_rejects(lib):
+    f = lib.dsa_sparse_mla_fwd
+    # null q
+    assert f(1, 0, 4, 16, 1, 576, 512, 0.1, None, 16, None, 8, None, 0, 0, None, 16, 4, 4, 16,
+             None, None, 0, None) == _lib.DSA_ERR_INVALID_ARG
+    # ld_idx < k_sel
+    assert f(1, 0, 4, 16, 1, 576, 512, 0.1, 16, 16, None, 8, None, 0, 0, None, 16, 4, 2, 16,
+             None, None, 0, None) == _lib.DSA_ERR_INVALID_ARG
+    # non-positive scale
+    assert f(1, 0, 4, 16, 1, 576, 512, 0.0, 16, 16, None, 8, None, 0, 0, None, 16, 4, 4, 16,
+             None, None, 0, None) == _lib.DSA_ERR_INVALID_ARG
+    # empty batch is a no-op
+    assert f(1, 0, 0, 16, 1, 576, 512, 0.1, 16, 16, None, 8, None, 0, 0, None, 16, 4, 4, 16,
+             None, None, 0, None) == _lib.DSA_OK
+
+
+def test_workspace_sizes(lib):
+    assert lib.dsa_sparse_mla_workspace_size(0, 100, 16, 512, 2048) == 0
+    ws = lib.dsa_sparse_mla_workspace_size(1, 64, 16, 512, 2048)
+    assert ws > 0 and ws % (64 * 16 * 513 * 4) == 0
+    assert lib.dsa_layer_stack_workspace_size(65536, 0) == 64 << 20
+    assert lib.dsa_layer_stack_workspace_size(1000, 0) == 1000 * 1000 * 4
+    assert lib.dsa_layer_stack_workspace_size(100, 16) == 16 * 100 * 4
+
+
+def test_launch_counters_reset(lib):
+    dsa.reset_launch_counts()
+    for k in range(4):
+        assert dsa.launch_count(k) == 0
+    assert dsa.launch_count(9) == -1
