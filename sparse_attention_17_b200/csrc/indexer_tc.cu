@@ -16,10 +16,11 @@
 // accumulator (2 x 256 columns), warp 2 owns the TMEM allocation, warps 4..11 drain the
 // accumulator: tcgen05.ld, ReLU, weight, reduce, causal mask, coalesced fp32 stores.
 //
-// Prefill units are blocks of 16 queries; their causal key range grows with the query
-// position, so persistent CTAs take units in snake order to even out the triangle.
-// Decode units are (sequence, 2048-key chunk); key tiles are assembled from pages with one
-// TMA load per page.
+// Work units are (query block, chunk of at most 32 key tiles): prefill blocks hold 16
+// queries and their causal key range grows with the query position, so the range is cut
+// into chunks to give every SM work even for a narrow window of query rows.  Decode units
+// are (sequence, 2048-key chunk); key tiles are assembled from pages with one TMA load per
+// page.  The query block and its head weights are double-buffered across units.
 #include "dsa_common.cuh"
 #include "launch.h"
 
@@ -36,15 +37,16 @@ constexpr int kEpiWarp0 = 4;       // first epilogue warp
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kTileBytes = kBM * 128;  // 128 keys x 64 bf16
 constexpr int kDecodeChunkTiles = 16;       // decode unit = 2048 keys
+constexpr int kPrefillChunkTiles = 32;      // prefill unit: at most 4096 keys
 
 template <int QB>
 struct IdxSmem {
     alignas(1024) uint8_t k[kStages][kTileBytes];
-    alignas(1024) uint8_t q[QB * kHI * 128 < 1024 ? 1024 : QB * kHI * 128];
-    float w[kEpiWarps][QB >= 2 ? QB / 2 * kHI : kHI];  // per-warp head weights of its queries
+    alignas(1024) uint8_t q[2][QB * kHI * 128 < 1024 ? 1024 : QB * kHI * 128];
+    alignas(16) float w[2][QB * kHI];  // head weights of the unit's queries
     uint64_t k_full[kStages];
     uint64_t k_empty[kStages];
-    uint64_t q_full, q_empty;
+    uint64_t q_full[2], q_empty[2];
     uint64_t acc_full[2], acc_empty[2];
     uint32_t tmem_base;
     int abort;
@@ -57,6 +59,8 @@ struct IdxParams {
     int q_begin, q_end;  // prefill query rows [q_begin, q_end)
     int S;               // prefill: key rows
     int num_units;
+    int nb;              // prefill: query blocks in the window
+    int nchunks;         // prefill: key chunks of the longest block
     // decode
     const int* page_table;
     const int* seq_lens;
@@ -78,15 +82,30 @@ struct UnitInfo {
     int len;        // decode: valid keys of the sequence
 };
 
+// Prefill: first query block whose causal key range reaches key chunk c.
+__host__ __device__ __forceinline__ int first_block_of_chunk(int c, int q_begin, int QB) {
+    const long long need = (long long)c * kPrefillChunkTiles * kBM - q_begin - QB + 1;
+    return need <= 0 ? 0 : (int)((need + QB - 1) / QB);
+}
+
 template <int QB, bool PAGED>
 __device__ __forceinline__ UnitInfo<QB, PAGED> unit_info(const IdxParams& p, int u) {
     UnitInfo<QB, PAGED> x;
     if constexpr (!PAGED) {
-        x.row0 = p.q_begin + u * QB;
+        // units are enumerated chunk by chunk: chunk c covers blocks first_block(c)..nb-1
+        int c = 0, rem = u, b = 0;
+        for (; c < p.nchunks; ++c) {
+            const int b0 = min(first_block_of_chunk(c, p.q_begin, QB), p.nb);
+            const int cnt = p.nb - b0;
+            if (rem < cnt) { b = b0 + rem; break; }
+            rem -= cnt;
+        }
+        x.row0 = p.q_begin + b * QB;
         const int t_max = min(x.row0 + QB, p.q_end) - 1;
-        x.tile0 = 0;
-        x.ntiles = t_max / kBM + 1;
-        x.len = 0;
+        const int total = t_max / kBM + 1;
+        x.tile0 = c * kPrefillChunkTiles;
+        x.ntiles = max(0, min(kPrefillChunkTiles, total - x.tile0));
+        x.len = min(x.row0 + QB, p.q_end) - x.row0;  // queries in the block
     } else {
         const int units_per_seq = (p.max_len + kBM * kDecodeChunkTiles - 1) / (kBM * kDecodeChunkTiles);
         x.row0 = u / units_per_seq;
@@ -123,8 +142,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(&sm.k_full[i], 1);
             mbar_init(&sm.k_empty[i], 1);
         }
-        mbar_init(&sm.q_full, 1);
-        mbar_init(&sm.q_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.q_full[i], 1);
+            mbar_init(&sm.q_empty[i], 1 + kEpiWarps);  // UMMA commit + epilogue warps
+        }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.acc_full[i], 1);
             mbar_init(&sm.acc_empty[i], kEpiWarps);
@@ -150,9 +171,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const int u = unit_at(i);
             if (u >= p.num_units) break;
             const UnitInfo<QB, PAGED> x = unit_info<QB, PAGED>(p, u);
-            if (!mbar_wait(&sm.q_empty, (ui & 1) ^ 1, abort, p.err)) break;
-            mbar_arrive_expect_tx(&sm.q_full, kQBytes);
-            tma_load_2d(sm.q, &tmap_q, 0, x.row0 * kHI, &sm.q_full);
+            const int qb = ui & 1;
+            if (!mbar_wait(&sm.q_empty[qb], ((ui >> 1) & 1) ^ 1, abort, p.err)) break;
+            // query block (TMA, swizzled) and its head weights (bulk copy) on one barrier
+            const int nq = PAGED ? 1 : x.len;
+            const uint32_t wbytes = (uint32_t)nq * kHI * 4;
+            mbar_arrive_expect_tx(&sm.q_full[qb], kQBytes + wbytes);
+            tma_load_2d(sm.q[qb], &tmap_q, 0, x.row0 * kHI, &sm.q_full[qb]);
+            bulk_load(sm.w[qb], p.w + (long long)x.row0 * kHI, wbytes, &sm.q_full[qb]);
             bool ok = true;
             for (int j = 0; j < x.ntiles; ++j, ++it) {
                 const int st = it % kStages;
@@ -182,13 +208,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- UMMA issuer ----------------
-        const uint32_t q_addr = smem_u32(sm.q);
         uint32_t it = 0;
         for (int i = 0, ui = 0;; ++i, ++ui) {
             const int u = unit_at(i);
             if (u >= p.num_units) break;
             const UnitInfo<QB, PAGED> x = unit_info<QB, PAGED>(p, u);
-            if (!mbar_wait(&sm.q_full, ui & 1, abort, p.err)) break;
+            const int qb = ui & 1;
+            if (!mbar_wait(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err)) break;
+            const uint32_t q_addr = smem_u32(sm.q[qb]);
             bool ok = true;
             for (int j = 0; j < x.ntiles; ++j, ++it) {
                 const int st = it % kStages;
@@ -206,7 +233,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 umma_commit(&sm.k_empty[st]);
                 umma_commit(&sm.acc_full[ab]);
             }
-            umma_commit(&sm.q_empty);
+            umma_commit(&sm.q_empty[qb]);
             if (!ok) break;
         }
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiWarps) {
@@ -221,16 +248,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const int u = unit_at(i);
             if (u >= p.num_units) break;
             const UnitInfo<QB, PAGED> x = unit_info<QB, PAGED>(p, u);
-            // this warp's queries' head weights (warp-private; no cross-warp barrier)
-            float* wbuf = sm.w[ew];
-            __syncwarp();
-            for (int e = lane; e < QPW * kHI; e += 32) {
-                const int qidx = half * QPW + e / kHI;
-                const int t = x.row0 + qidx;
-                const bool valid = active_half && (PAGED ? true : (t < p.q_end));
-                wbuf[e] = valid ? __ldg(p.w + (long long)t * kHI + (e % kHI)) : 0.f;
-            }
-            __syncwarp();
+            const int qb = ui & 1;
+            if (!mbar_wait(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err)) break;
+            const float* wbuf = sm.w[qb] + half * QPW * kHI;  // this warp's queries' weights
             bool ok = true;
             for (int j = 0; j < x.ntiles; ++j, ++it) {
                 const int ab = it & 1;
@@ -264,7 +284,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                             const float score = acc0 + acc1;
                             if constexpr (!PAGED) {
                                 const int t = x.row0 + qidx;
-                                if (t < p.q_end && s <= t)
+                                if (qidx < x.len && s <= t)
                                     p.scores[(long long)(t - p.q_begin) * p.ld + s] = score;
                             } else {
                                 if (s < x.len) p.scores[(long long)x.row0 * p.ld + s] = score;
@@ -277,6 +297,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
             }
             if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.q_empty[qb]);  // done with this unit's weights
         }
     }
 
@@ -324,7 +346,17 @@ cudaError_t launch_indexer_bf16_prefill(const __nv_bfloat16* q_idx, const __nv_b
     p.q_begin = q_begin;
     p.q_end = q_begin + rows;
     p.S = S;
-    p.num_units = (rows + QB - 1) / QB;
+    p.nb = (rows + QB - 1) / QB;
+    {
+        const int t_max = q_begin + rows - 1;
+        p.nchunks = (t_max / kBM + 1 + kPrefillChunkTiles - 1) / kPrefillChunkTiles;
+        long long units = 0;
+        for (int c = 0; c < p.nchunks; ++c) {
+            int b0 = first_block_of_chunk(c, q_begin, QB);
+            units += p.nb - (b0 < p.nb ? b0 : p.nb);
+        }
+        p.num_units = (int)units;
+    }
     p.err = ctx.err;
     const int grid = p.num_units < ctx.num_sms ? p.num_units : ctx.num_sms;
     return launch_indexer_tc<QB, false>(tq, tk, p, grid, stream);

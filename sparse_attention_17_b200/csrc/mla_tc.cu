@@ -62,7 +62,7 @@ struct MlaSmem {
     alignas(1024) uint8_t q[2][kQBytes];
     alignas(1024) uint8_t p[2][kPBytes];
     float red[2][4][kH];
-    float lred[4][kH];
+    float lred[8][kH];
     uint64_t a_full[2], s_full[2], p_full[2], pv_done[2];
     uint64_t q_full[2], q_empty[2];
     uint64_t o_free;
@@ -304,9 +304,11 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
             const int u = blockIdx.x + ui * gridDim.x;
             if (u >= p.num_units) break;
             const Unit x = unit_of(p, u);
-            float m_ref[kH], l_part[kH];
+            // l_part: sums of the bf16 probabilities fed to the PV product (normalises O);
+            // l_lse: the same sums before rounding (for the log-sum-exp output)
+            float m_ref[kH], l_part[kH], l_lse[kH];
 #pragma unroll
-            for (int h = 0; h < kH; ++h) { m_ref[h] = -INFINITY; l_part[h] = 0.f; }
+            for (int h = 0; h < kH; ++h) { m_ref[h] = -INFINITY; l_part[h] = 0.f; l_lse[h] = 0.f; }
             bool ok = true;
             for (int j = 0; j < x.nb; ++j, ++G) {
                 const int s = G & 1;
@@ -368,7 +370,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
                     }
                     tmem_wait_st();
 #pragma unroll
-                    for (int h = 0; h < kH; ++h) l_part[h] *= alpha[h];
+                    for (int h = 0; h < kH; ++h) { l_part[h] *= alpha[h]; l_lse[h] *= alpha[h]; }
                 }
                 // P buffer s is free once the PV product of block G-2 has completed
                 if (!mbar_wait(&sm.pv_done[s], ph ^ 1, abort, p.err)) { ok = false; break; }
@@ -379,6 +381,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
                         const float pv = valid ? exp2f(xs[h] - m_ref[h]) : 0.f;
                         const __nv_bfloat16 b = __float2bfloat16_rn(pv);
                         l_part[h] += __bfloat162float(b);
+                        l_lse[h] += pv;
                         const int off = (h >> 3) * 1024 + (h & 7) * 128 +
                                         ((((2 * r) >> 4) ^ (h & 7)) << 4) + ((2 * r) & 15);
                         *reinterpret_cast<__nv_bfloat16*>(pb + off) = b;
@@ -392,7 +395,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
             if (!ok) break;
 
             // -------- epilogue of this unit --------
-            float L[kH];
+            float L[kH], Lx[kH];
             if (x.nb > 0) {
                 const uint32_t Gp = G - 1;
                 if (!mbar_wait(&sm.pv_done[Gp & 1], (Gp >> 1) & 1, abort, p.err)) break;
@@ -404,18 +407,25 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
                     v += __shfl_xor_sync(0xffffffffu, v, 4);
                     v += __shfl_xor_sync(0xffffffffu, v, 2);
                     v += __shfl_xor_sync(0xffffffffu, v, 1);
-                    if (lane == 0) sm.lred[quad][h] = v;
+                    float e = l_lse[h];
+                    e += __shfl_xor_sync(0xffffffffu, e, 8);
+                    e += __shfl_xor_sync(0xffffffffu, e, 4);
+                    e += __shfl_xor_sync(0xffffffffu, e, 2);
+                    e += __shfl_xor_sync(0xffffffffu, e, 1);
+                    if (lane == 0) { sm.lred[quad][h] = v; sm.lred[4 + quad][h] = e; }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.epi_bar);
                 if (!mbar_wait(&sm.epi_bar, epi_phase, abort, p.err)) break;
                 epi_phase ^= 1;
 #pragma unroll
-                for (int h = 0; h < kH; ++h)
+                for (int h = 0; h < kH; ++h) {
                     L[h] = sm.lred[0][h] + sm.lred[1][h] + sm.lred[2][h] + sm.lred[3][h];
+                    Lx[h] = sm.lred[4][h] + sm.lred[5][h] + sm.lred[6][h] + sm.lred[7][h];
+                }
             } else {
 #pragma unroll
-                for (int h = 0; h < kH; ++h) L[h] = 0.f;
+                for (int h = 0; h < kH; ++h) { L[h] = 0.f; Lx[h] = 0.f; }
             }
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
@@ -435,10 +445,10 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
                 }
             }
             if (quad == 0 && lane < kH) {
-                float mr = m_ref[0], Lh = L[0];
+                float mr = m_ref[0], Lh = Lx[0];
 #pragma unroll
                 for (int h = 1; h < kH; ++h)
-                    if (lane == h) { mr = m_ref[h]; Lh = L[h]; }
+                    if (lane == h) { mr = m_ref[h]; Lh = Lx[h]; }
                 const float l = Lh > 0.f ? (mr + log2f(Lh)) * 0.69314718055994531f : -INFINITY;
                 if (p.page_table == nullptr) {
                     if (p.lse != nullptr) p.lse[(long long)x.n * kH + lane] = l;

@@ -5,18 +5,20 @@
 // n <= k every key is selected.  Output: the selected key positions in ascending order,
 // then -1 padding.
 //
-// One CTA of 512 threads per row.  Scores map to order-preserving uint32 keys and the
-// k-th largest key (tau) is found one radix digit at a time (12 + 12 + 8 bits):
-//   pass 1  (global read)  histogram of bits 31..20 -> digit b1 holding the k-th key;
-//   pass 2  (global read)  keys with digit > b1 are selected (a bitmap word per warp
-//           ballot); keys with digit == b1 are appended to a candidate list in shared
-//           memory;
-//   refine  (shared memory) two more digit histograms over the candidates give tau;
-//           candidates above tau are selected, those equal to tau marked as ties.
-// If the b1 bucket is larger than the candidate buffer, the refinement reads the row
-// from global memory again instead (correct for any input, e.g. all scores equal).
-// Finally the first `need` ties in index order are kept and the bitmap is compacted in
-// index order, which yields ascending indices without sorting.
+// One CTA of 512 threads per row.  Scores map to order-preserving uint32 keys.
+// Fast path (one read of the row):
+//   sample  every 16th 32-key chunk of the row goes to shared memory; an exact radix
+//           select there picks a provisional threshold tau0 a few standard deviations
+//           below the sample's k-th-largest-equivalent rank (rows of at most 8192 keys
+//           skip this: tau0 = the smallest key);
+//   gather  one vectorised pass appends every key >= tau0 to a shared candidate list
+//           (warp ballots, one shared atomic per warp);
+//   select  radix select (12 + 12 + 8 bits) among the candidates gives the k-th largest
+//           key tau; candidates above tau are selected, those equal to tau are ties.
+// If the candidates number fewer than k or more than the buffer holds, the row is redone
+// exactly from global memory (histogram passes over the whole row).  Finally the first
+// `need` ties in index order are kept and a bitmap of the selection is compacted in index
+// order, which yields ascending indices without sorting.
 #include "dsa_common.cuh"
 #include "launch.h"
 
@@ -39,6 +41,8 @@ struct TopkScratch {
     uint32_t found_bin;
     uint32_t found_above;
 };
+
+constexpr int kSampleChunks = kCandCap / 32;  // at most 256 sampled 32-key chunks
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
@@ -111,39 +115,56 @@ __device__ __forceinline__ void zero_hist(TopkScratch& sh, int nbins) {
     for (int i = threadIdx.x; i < nbins; i += kThreads) sh.hist[i] = 0u;
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
-topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
-                  const int* __restrict__ row_len, int max_len, int k, int* __restrict__ idx,
-                  long long ld_idx, unsigned* __restrict__ err) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    TopkScratch& sh = *reinterpret_cast<TopkScratch*>(smem_raw);
-    uint32_t* sel = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkScratch));
-    const int max_words = (max_len + 31) >> 5;
-    uint32_t* tie = sel + max_words;
-
-    const int r = blockIdx.x;
+// Exact radix select of the `need`-th largest of keys[0..cnt) (shared memory): returns the
+// key value tau; *need_out = how many keys equal to tau belong to the top `need`.
+__device__ uint32_t smem_radix_select(TopkScratch& sh, const uint32_t* keys, int cnt,
+                                      uint32_t need, uint32_t* need_out) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int n;
-    if (row_len != nullptr) {
-        n = row_len[r];
-        if (n < 0 || n > max_len) {
-            if (threadIdx.x == 0) atomicOr(err, DSA_DEVERR_INDEX_RANGE);
-            n = n < 0 ? 0 : max_len;
-        }
-    } else {
-        n = q_begin + r + 1;
+    zero_hist(sh, kBins);
+    __syncthreads();
+    for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
+        const int c = c0 + lane;
+        hist_add(sh.hist, c < cnt ? keys[c] >> 20 : 0u, c < cnt);
     }
-    int* out = idx + (long long)r * ld_idx;
-    if (n <= k) {  // every valid key is selected
-        for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
-        return;
+    __syncthreads();
+    find_bin(sh, kBins, need);
+    const uint32_t b1 = sh.found_bin;
+    need -= sh.found_above;
+    zero_hist(sh, kBins);
+    __syncthreads();
+    for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
+        const int c = c0 + lane;
+        const uint32_t key = c < cnt ? keys[c] : 0u;
+        hist_add(sh.hist, (key >> 8) & 0xFFFu, c < cnt && (key >> 20) == b1);
     }
-    const float* row = scores + (long long)r * ld;
-    const int nwords = (n + 31) >> 5;
+    __syncthreads();
+    find_bin(sh, kBins, need);
+    const uint32_t pre = (b1 << 12) | sh.found_bin;
+    need -= sh.found_above;
+    zero_hist(sh, 256);
+    __syncthreads();
+    for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
+        const int c = c0 + lane;
+        const uint32_t key = c < cnt ? keys[c] : 0u;
+        hist_add(sh.hist, key & 0xFFu, c < cnt && (key >> 8) == pre);
+    }
+    __syncthreads();
+    find_bin(sh, 256, need);
+    need -= sh.found_above;
+    *need_out = need;
+    const uint32_t tau = (pre << 8) | sh.found_bin;
+    __syncthreads();
+    return tau;
+}
 
+// Exact selection from global memory (fallback): histogram passes over the whole row.
+// Fills sel (keys above the k-th largest) and tie (keys equal to it); returns how many
+// of the ties belong to the top k.  sel must be zero, tie zero on entry.
+__device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ row, int n,
+                                     int k, uint32_t* sel, uint32_t* tie) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // ---- pass 1: histogram of the top 12 key bits over the whole row ----
     zero_hist(sh, kBins);
-    for (int i = threadIdx.x; i < nwords; i += kThreads) tie[i] = 0u;
     if (threadIdx.x == 0) sh.cand_count = 0u;
     __syncthreads();
     for (int base = warp * 32; base < n; base += 4 * kStride) {
@@ -259,6 +280,113 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
                 tie[base >> 5] = eq;
             }
         }
+    }
+    __syncthreads();
+    return need;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
+                  const int* __restrict__ row_len, int max_len, int k, int* __restrict__ idx,
+                  long long ld_idx, unsigned* __restrict__ err) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    TopkScratch& sh = *reinterpret_cast<TopkScratch*>(smem_raw);
+    uint32_t* sel = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkScratch));
+    const int max_words = (max_len + 31) >> 5;
+    uint32_t* tie = sel + max_words;
+
+    const int r = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int n;
+    if (row_len != nullptr) {
+        n = row_len[r];
+        if (n < 0 || n > max_len) {
+            if (threadIdx.x == 0) atomicOr(err, DSA_DEVERR_INDEX_RANGE);
+            n = n < 0 ? 0 : max_len;
+        }
+    } else {
+        n = q_begin + r + 1;
+    }
+    int* out = idx + (long long)r * ld_idx;
+    if (n <= k) {  // every valid key is selected
+        for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    const float* row = scores + (long long)r * ld;
+    const int nwords = (n + 31) >> 5;
+    for (int i = threadIdx.x; i < nwords; i += kThreads) tie[i] = 0u;
+    if (threadIdx.x == 0) sh.cand_count = 0u;
+    __syncthreads();
+
+    // ---- provisional threshold from a sample of the row ----
+    uint32_t tau0 = 0u;
+    if (n > kCandCap) {
+        const int nchunks = (n + 31) >> 5;
+        const int stride = max(16, (nchunks + kSampleChunks - 1) / kSampleChunks);
+        const int nsamp = (nchunks + stride - 1) / stride;  // sampled chunks
+        uint32_t valid = 0;
+        for (int j = warp; j < nsamp; j += kWarps) {
+            const int sidx = j * stride * 32 + lane;
+            const bool in = sidx < n;
+            sh.cand_key[j * 32 + lane] = in ? float_order_key(__ldg(row + sidx)) : 0u;
+            valid += __popc(__ballot_sync(0xffffffffu, in));
+        }
+        if (lane == 0) atomicAdd(&sh.cand_count, valid);
+        __syncthreads();
+        const uint32_t m = sh.cand_count;
+        // rank in the sample whose key should leave >= k keys of the row above it
+        const float expect = (float)k * (float)m / (float)n;
+        uint32_t rank = (uint32_t)ceilf(expect + 3.f * sqrtf(expect)) + 2u;
+        if (rank > m) rank = m;
+        uint32_t dummy;
+        tau0 = smem_radix_select(sh, sh.cand_key, nsamp * 32, rank, &dummy);
+        if (threadIdx.x == 0) sh.cand_count = 0u;
+        __syncthreads();
+    }
+
+    // ---- one pass: every key >= tau0 becomes a candidate ----
+    for (int base = warp * 128; base < n; base += kWarps * 128) {
+        const int s0 = base + 4 * lane;
+        float x[4];
+        if (s0 + 3 < n) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(row + s0));
+            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) x[u] = s0 + u < n ? __ldg(row + s0 + u) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint32_t key = float_order_key(x[u]);
+            const bool take = s0 + u < n && key >= tau0;
+            const unsigned m = __ballot_sync(0xffffffffu, take);
+            if (m) {
+                uint32_t pos0 = 0;
+                if (lane == 0) pos0 = atomicAdd(&sh.cand_count, (uint32_t)__popc(m));
+                pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+                const uint32_t p = pos0 + __popc(m & lanemask_lt());
+                if (take && p < (uint32_t)kCandCap) {
+                    sh.cand_key[p] = key;
+                    sh.cand_idx[p] = s0 + u;
+                }
+            }
+        }
+    }
+    for (int i = threadIdx.x; i < nwords; i += kThreads) sel[i] = 0u;
+    __syncthreads();
+    const uint32_t ncand = sh.cand_count;
+    __syncthreads();  // everyone has read the count before it can be reused
+    uint32_t need;
+    if (ncand >= (uint32_t)k && ncand <= (uint32_t)kCandCap) {
+        const uint32_t tau = smem_radix_select(sh, sh.cand_key, (int)ncand, (uint32_t)k, &need);
+        for (int c = threadIdx.x; c < (int)ncand; c += kThreads) {
+            const uint32_t key = sh.cand_key[c];
+            const int sidx = sh.cand_idx[c];
+            if (key > tau) atomicOr(&sel[sidx >> 5], 1u << (sidx & 31));
+            else if (key == tau) atomicOr(&tie[sidx >> 5], 1u << (sidx & 31));
+        }
+    } else {
+        need = exact_row_select(sh, row, n, k, sel, tie);
     }
     __syncthreads();
 

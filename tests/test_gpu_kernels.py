@@ -243,3 +243,19 @@ def test_deterministic_reruns():
         outs.append((idx.cpu(), out.cpu()))
     assert torch.equal(outs[0][0], outs[1][0])
     assert torch.equal(outs[0][1].view(torch.int16), outs[1][1].view(torch.int16))
+
+
+def test_topk_sample_miss_falls_back_to_exact():
+    """The large scores sit only in 32-key chunks the threshold sample never reads, so the
+    provisional threshold admits too many candidates; the exact path must take over."""
+    S, k = 40960, 2048
+    sc = np.zeros((2, S))
+    chunks = np.arange(S // 32)
+    hot = chunks[chunks % 16 != 0]
+    r = np.random.default_rng(9)
+    for c in hot[: 2 * k // 32]:
+        sc[0, c * 32:(c + 1) * 32] = r.normal(10, 1, 32)
+    sc[1] = r.normal(size=S)
+    sc[1, ::512] = 50.0  # sampled chunk heads are huge: threshold too high, too few candidates
+    idx, ref = _topk_case(sc, [S, S], k, row_len=True)
+    check_indices_exact(idx, ref, "sample miss")
