@@ -65,6 +65,30 @@ def algorithmic_work(T, k):
     }
 
 
+def shard_plan(rank, world, T, k):
+    """Weak scaling over independent sequences: rank r prefills its own length-T sequence
+    (inputs seeded r); nothing crosses ranks on the data path."""
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    return {"seed": rank, "T": T, "topk": k, "tokens": T}
+
+
+def max_over_ranks(x, device=None):
+    """Max of a per-rank float over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tokens_per_s(tokens_per_rank, world, ms_per_step):
+    """Whole-job throughput: all ranks' tokens over the slowest rank's step time."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def load_peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -189,8 +213,9 @@ def run_native(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    T, k = args.T, args.topk
-    host = make_inputs(T, k, seed=rank)
+    plan = shard_plan(rank, world, args.T, args.topk)
+    T, k = plan["T"], plan["topk"]
+    host = make_inputs(T, k, seed=plan["seed"])
     names = ("q_idx", "k_idx", "w", "q", "kv")
     x = {n: host[n].to(dev) for n in names}
     ld = (T + 3) // 4 * 4
@@ -243,10 +268,7 @@ def run_native(args, rank, world, local_rank):
     idx_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     mla_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     errs = dsa.check_device_errors()
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dev)
 
     # per-kernel split of the index phase (separate, untimed-for-value pass)
     e_idx = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(windows) + 1)]
@@ -285,11 +307,9 @@ def run_native(args, rank, world, local_rank):
         t2.record(stream)
         torch.cuda.synchronize()
         e2e_ms = s2.elapsed_time(t2) / n_e2e
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e_ms = max_over_ranks(e2e_ms, dev)
+        e2e = {"value": aggregate_tokens_per_s(T, world, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     result = None
@@ -297,7 +317,7 @@ def run_native(args, rank, world, local_rank):
         work = algorithmic_work(T, k)
         peaks, peak_src = load_peaks()
         ms_step = ms_total / args.steps
-        value = world * T / (ms_step / 1e3)
+        value = aggregate_tokens_per_s(T, world, ms_step)
         kern = {"indexer_ms": indexer_ms, "topk_ms": topk_ms, "sparse_mla_ms": mla_ms,
                 "index_phase_ms": idx_ms}
         # dominant kernel

@@ -275,6 +275,9 @@ dsa_status dsa_sparse_mla_fwd(int dtype, int mode, int num_q, int H, int num_kv_
     if (H != 16 || num_kv_heads != 1 || D_qk != 576 || D_v != 512 || v != nullptr)
         return fail(DSA_ERR_UNSUPPORTED,
                     "bf16 path is absorbed MLA: H=16, one shared 576-dim latent, D_v=512, v=NULL");
+    if (k_sel > 2048 || (k_sel & 3) || (ld_idx & 3))
+        return fail(DSA_ERR_UNSUPPORTED,
+                    "bf16 MLA path: k_sel <= 2048 and k_sel, ld_idx multiples of 4");
     if (mode == DSA_PREFILL) {
         if (page_table || seq_lens) return fail(DSA_ERR_INVALID_ARG, "prefill takes no pages");
         e = launch_sparse_mla_bf16(static_cast<const __nv_bfloat16*>(q),

@@ -77,13 +77,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           unsigned* err) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
-    while (true) {
+    for (uint32_t spin = 1;; ++spin) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-            atomicOr(err, DSA_DEVERR_TIMEOUT);
-            *abort = 1;
-            return false;
+        if ((spin & 15u) == 0u) {  // the timer and the abort flag are polled rarely
+            if (*abort) return false;
+            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+                atomicOr(err, DSA_DEVERR_TIMEOUT);
+                *abort = 1;
+                return false;
+            }
         }
     }
 }
@@ -121,6 +123,14 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, 
 // ------------------------------------------------------------------------------------
 __device__ __forceinline__ void cp_async_16(uint32_t smem_dst, const void* gmem_src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gmem_src)
+                 : "memory");
+}
+
+// 16 zero bytes to shared memory through the same asynchronous path (src-size 0: nothing
+// is read from `any_global`, which only has to be a valid address).
+__device__ __forceinline__ void cp_async_16_zero(uint32_t smem_dst, const void* any_global) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, 0;" ::"r"(smem_dst),
+                 "l"(any_global)
                  : "memory");
 }
 

@@ -49,9 +49,10 @@ constexpr int kThreads = 288;
 constexpr int kMmaWarp = 4;
 constexpr int kGatherWarp0 = 5;
 constexpr int kGatherThreads = 128;
+constexpr int kIdxCap = 2048;                 // index entries of one unit held in smem
 constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t kOCol = 0;                 // O^T: 4 M-tiles x 16 columns
-constexpr uint32_t kSCol = 64;                // S^T stage s at kSCol + 16 s
+constexpr uint32_t kSCol = 64;                // S^T of stage s at kSCol + 16 s
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(64, kH, 0, 0);
@@ -61,7 +62,8 @@ struct MlaSmem {
     alignas(1024) uint8_t a[2][kStageBytes];
     alignas(1024) uint8_t q[2][kQBytes];
     alignas(1024) uint8_t p[2][kPBytes];
-    float red[2][4][kH];
+    alignas(16) int idx[2][kIdxCap];  // the unit's selected indices (bulk-copied with Q)
+    alignas(16) float red[2][4][kH];
     float lred[8][kH];
     uint64_t a_full[2], s_full[2], p_full[2], pv_done[2];
     uint64_t q_full[2], q_empty[2];
@@ -122,11 +124,12 @@ __device__ __forceinline__ Unit unit_of(const MlaParams& p, int u) {
 }
 
 // Row of the latent cache for index entry e of unit x, or -1 (padding / invalid).
-// Out-of-range entries are recorded in the error word when `report` is set.
-__device__ __forceinline__ long long resolve_row(const MlaParams& p, const Unit& x, int e,
-                                                 bool report) {
+// `uidx` holds the unit's entries e0..e1-1 (shared memory).  Out-of-range entries are
+// recorded in the error word when `report` is set.
+__device__ __forceinline__ long long resolve_row(const MlaParams& p, const Unit& x,
+                                                 const int* uidx, int e, bool report) {
     if (e >= x.e1) return -1;
-    const int s = __ldg(p.idx + (long long)x.n * p.ld_idx + e);
+    const int s = uidx[e - x.e0];
     if (s < 0) return -1;
     if (p.page_table == nullptr) {
         if (s >= p.kv_rows) {
@@ -147,6 +150,11 @@ __device__ __forceinline__ long long resolve_row(const MlaParams& p, const Unit&
     return (long long)pg * p.page_size + s % p.page_size;
 }
 
+// Inverse of float_order_key.
+__device__ __forceinline__ float order_key_to_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -162,7 +170,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
             mbar_init(&sm.p_full[i], 4);
             mbar_init(&sm.pv_done[i], 1);
             mbar_init(&sm.q_full[i], 1);
-            mbar_init(&sm.q_empty[i], 1);
+            mbar_init(&sm.q_empty[i], 1 + 4 + 4);  // UMMA commit + gather + softmax warps
         }
         mbar_init(&sm.o_free, 4);
         mbar_init(&sm.red_bar[0], 4);
@@ -185,6 +193,28 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
         const int gw = warp - kGatherWarp0;  // keys gw*16 .. gw*16+15 of each block
         const bool q_leader = (gw == 0 && lane == 0);
         if (q_leader) tma_prefetch_desc(&tmap_q);
+        // The leader issues each unit's query (TMA) and index entries (bulk copy) into the
+        // double buffer as soon as the buffer is free, one unit ahead where possible.
+        int issued = 0;
+        auto issue_unit_loads = [&](bool blocking) {
+            const int u2 = blockIdx.x + issued * gridDim.x;
+            if (u2 >= p.num_units) return;
+            const int qb2 = issued & 1;
+            const uint32_t par = ((issued >> 1) & 1) ^ 1;
+            const bool free = blocking ? mbar_wait(&sm.q_empty[qb2], par, abort, p.err)
+                                       : mbar_try_wait(&sm.q_empty[qb2], par);
+            if (!free) return;
+            const Unit y = unit_of(p, u2);
+            const uint32_t ibytes = (uint32_t)(y.e1 - y.e0) * 4u;
+            mbar_arrive_expect_tx(&sm.q_full[qb2], kQBytes + ibytes);
+            for (int c = 0; c < kChunks; ++c)
+                tma_load_2d(sm.q[qb2] + c * kQChunkBytes, &tmap_q, c * 64, y.n * kH,
+                            &sm.q_full[qb2]);
+            if (ibytes)
+                bulk_load(sm.idx[qb2], p.idx + (long long)y.n * p.ld_idx + y.e0, ibytes,
+                          &sm.q_full[qb2]);
+            ++issued;
+        };
         uint32_t G = 0;
         for (int ui = 0;; ++ui) {
             const int u = blockIdx.x + ui * gridDim.x;
@@ -192,43 +222,44 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
             const Unit x = unit_of(p, u);
             const int qb = ui & 1;
             if (q_leader) {
-                if (mbar_wait(&sm.q_empty[qb], ((ui >> 1) & 1) ^ 1, abort, p.err)) {
-                    mbar_arrive_expect_tx(&sm.q_full[qb], kQBytes);
-                    for (int c = 0; c < kChunks; ++c)
-                        tma_load_2d(sm.q[qb] + c * kQChunkBytes, &tmap_q, c * 64, x.n * kH,
-                                    &sm.q_full[qb]);
-                }
+                while (issued <= ui && !*abort) issue_unit_loads(true);
+                issue_unit_loads(false);  // prefetch the next unit if its buffer is free
             }
+            if (!mbar_wait(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err)) break;
+            const int* uidx = sm.idx[qb];
             bool ok = true;
             for (int j = 0; j < x.nb; ++j, ++G) {
                 const int s = G & 1;
                 const uint32_t ph = (G >> 1) & 1;
                 if (!mbar_wait(&sm.pv_done[s], ph ^ 1, abort, p.err)) { ok = false; break; }
                 long long row = -1;
-                if (lane < 16) row = resolve_row(p, x, x.e0 + j * kBK + gw * 16 + lane, true);
-                const __nv_bfloat16* rptr = row >= 0 ? p.kv + row * kDqk : nullptr;
-                const uint32_t a_base = smem_u32(sm.a[s]);
+                if (lane < 16) row = resolve_row(p, x, uidx, x.e0 + j * kBK + gw * 16 + lane, true);
+                // lane l copies the 16-byte units l, l+32 and (l < 8) l+64 of each of the warp's
+                // 16 rows; unit u of row r goes to chunk u/8, line r, slot (u%8) ^ (r%8)
+                const uint32_t a_lane = smem_u32(sm.a[s]) + (lane >> 3) * kChunkBytes;
+                const char* kvb = reinterpret_cast<const char*>(p.kv) + lane * 16;
 #pragma unroll 4
-                for (int i = 0; i < 36; ++i) {
-                    const int f = i * 32 + lane;      // 16 keys x 72 units of 16 B
-                    const int kl = f / 72;
-                    const int unit = f - kl * 72;
-                    const __nv_bfloat16* src =
-                        reinterpret_cast<const __nv_bfloat16*>(__shfl_sync(0xffffffffu,
-                            reinterpret_cast<uintptr_t>(rptr), kl));
+                for (int kl = 0; kl < 16; ++kl) {
+                    const long long rr = __shfl_sync(0xffffffffu, row, kl);
                     const int r = gw * 16 + kl;
-                    const int c = unit >> 3, u8 = unit & 7;
-                    const uint32_t dst = a_base + c * kChunkBytes + r * 128 + ((u8 ^ (r & 7)) << 4);
-                    if (src != nullptr) {
-                        cp_async_16(dst, src + unit * 8);
+                    const uint32_t dst = a_lane + r * 128 + (((lane & 7) ^ (r & 7)) << 4);
+                    if (rr >= 0) {
+                        const char* src = kvb + rr * (kDqk * 2);
+                        cp_async_16(dst, src);
+                        cp_async_16(dst + 4 * kChunkBytes, src + 512);
+                        if (lane < 8) cp_async_16(dst + 8 * kChunkBytes, src + 1024);
                     } else {
-                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, 0;" ::"r"(dst),
-                                     "l"(p.kv) : "memory");
+                        cp_async_16_zero(dst, p.kv);
+                        cp_async_16_zero(dst + 4 * kChunkBytes, p.kv);
+                        if (lane < 8) cp_async_16_zero(dst + 8 * kChunkBytes, p.kv);
                     }
                 }
                 cp_async_mbar_arrive(&sm.a_full[s]);
+                if (q_leader && issued == ui + 1) issue_unit_loads(false);
             }
             if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.q_empty[qb]);  // done with this unit's indices
         }
         // let this thread's copies land before the CTA can exit
         asm volatile("cp.async.wait_all;" ::: "memory");
@@ -237,26 +268,43 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
         if (lane == 0) {
             uint32_t G = 0;
             int units_with_blocks = 0;
-            auto issue_pv = [&](uint32_t Gp, bool first, int prior_units) -> bool {
+            // Descriptors are built once; per UMMA only a constant start-address offset
+            // (in 16-byte units) is added.
+            // (stage 1 / buffer 1 follow stage 0 / buffer 0 at a fixed distance)
+            const uint64_t a_desc_k0 = smem_desc(smem_u32(sm.a[0]), 16, 1024, kSwizzle128B);
+            const uint64_t a_desc_mn0 = smem_desc(smem_u32(sm.a[0]), kChunkBytes, 1024, kSwizzle128B);
+            const uint64_t q_desc0 = smem_desc(smem_u32(sm.q[0]), 16, 1024, kSwizzle128B);
+            const uint64_t p_desc0 = smem_desc(smem_u32(sm.p[0]), 16, 1024, kSwizzle128B);
+            constexpr uint32_t kAStep = (uint32_t)(sizeof(MlaSmem::a[0]) >> 4);
+            constexpr uint32_t kQStep = (uint32_t)(sizeof(MlaSmem::q[0]) >> 4);
+            constexpr uint32_t kPStep = (uint32_t)(sizeof(MlaSmem::p[0]) >> 4);
+            auto issue_pv_now = [&](uint32_t Gp, bool first) {
                 const int s = Gp & 1;
-                const uint32_t ph = (Gp >> 1) & 1;
-                if (!mbar_wait(&sm.p_full[s], ph, abort, p.err)) return false;
-                if (first && prior_units > 0)
-                    if (!mbar_wait(&sm.o_free, (prior_units - 1) & 1, abort, p.err)) return false;
                 tc_fence_after();
-                const uint32_t a_base = smem_u32(sm.a[s]);
-                const uint32_t p_base = smem_u32(sm.p[s]);
+                // K-step outer, M-tile inner: consecutive UMMAs go to different accumulators
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
+                for (int kk = 0; kk < kBK / 16; ++kk) {
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-                        const uint64_t ad = smem_desc(a_base + 2 * m * kChunkBytes + kk * 2048,
-                                                      kChunkBytes, 1024, kSwizzle128B);
-                        const uint64_t bd = smem_desc(p_base + kk * 32, 16, 1024, kSwizzle128B);
-                        umma_bf16(tmem + kOCol + 16 * m, ad, bd, kIdescPV, !(first && kk == 0));
-                    }
+                    for (int m = 0; m < 4; ++m)
+                        umma_bf16(tmem + kOCol + 16 * m,
+                                  a_desc_mn0 + s * kAStep + ((2 * m * kChunkBytes + kk * 2048) >> 4),
+                                  p_desc0 + s * kPStep + ((kk * 32) >> 4), kIdescPV,
+                                  !(first && kk == 0));
                 }
                 umma_commit(&sm.pv_done[s]);
+            };
+            // PV of block Gp may start once its P is in smem (and, for the first block of
+            // a unit, once the previous unit's epilogue has read O out of TMEM).
+            auto pv_ready = [&](uint32_t Gp, bool first, int prior_units) -> bool {
+                if (!mbar_try_wait(&sm.p_full[Gp & 1], (Gp >> 1) & 1)) return false;
+                return !(first && prior_units > 0) ||
+                       mbar_try_wait(&sm.o_free, (prior_units - 1) & 1);
+            };
+            auto issue_pv = [&](uint32_t Gp, bool first, int prior_units) -> bool {
+                if (!mbar_wait(&sm.p_full[Gp & 1], (Gp >> 1) & 1, abort, p.err)) return false;
+                if (first && prior_units > 0)
+                    if (!mbar_wait(&sm.o_free, (prior_units - 1) & 1, abort, p.err)) return false;
+                issue_pv_now(Gp, first);
                 return true;
             };
             bool ok = true;
@@ -266,25 +314,39 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
                 const Unit x = unit_of(p, u);
                 const int qb = ui & 1;
                 if (!mbar_wait(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err)) break;
-                const uint32_t q_base = smem_u32(sm.q[qb]);
                 for (int j = 0; j < x.nb; ++j, ++G) {
                     const int s = G & 1;
                     const uint32_t ph = (G >> 1) & 1;
+                    // While block G's gather is in flight, start PV of block G-1 if its P is
+                    // ready, so that stage G-1 is released as early as possible.
+                    bool pv_prev_issued = j == 0;
+                    if (!pv_prev_issued) {
+                        for (uint32_t spin = 0; !mbar_try_wait(&sm.a_full[s], ph); ++spin) {
+                            if (pv_ready(G - 1, j - 1 == 0, units_with_blocks)) {
+                                issue_pv_now(G - 1, j - 1 == 0);
+                                pv_prev_issued = true;
+                                break;
+                            }
+                            if ((spin & 1023u) == 1023u && *abort) { ok = false; break; }
+                        }
+                        if (!ok) break;
+                    }
                     if (!mbar_wait(&sm.a_full[s], ph, abort, p.err)) { ok = false; break; }
                     fence_proxy_async_smem();
                     tc_fence_after();
-                    const uint32_t a_base = smem_u32(sm.a[s]);
 #pragma unroll
                     for (int kk = 0; kk < kDqk / 16; ++kk) {
                         const int c = kk >> 2, sub = kk & 3;
-                        const uint64_t ad = smem_desc(a_base + c * kChunkBytes + sub * 32, 16,
-                                                      1024, kSwizzle128B);
-                        const uint64_t bd = smem_desc(q_base + c * kQChunkBytes + sub * 32, 16,
-                                                      1024, kSwizzle128B);
-                        umma_bf16(tmem + kSCol + 16 * s, ad, bd, kIdescQK, kk > 0);
+                        umma_bf16(tmem + kSCol + 16 * s,
+                                  a_desc_k0 + s * kAStep + ((c * kChunkBytes + sub * 32) >> 4),
+                                  q_desc0 + qb * kQStep + ((c * kQChunkBytes + sub * 32) >> 4),
+                                  kIdescQK, kk > 0);
                     }
                     umma_commit(&sm.s_full[s]);
-                    if (j >= 1 && !issue_pv(G - 1, j - 1 == 0, units_with_blocks)) { ok = false; break; }
+                    if (!pv_prev_issued && !issue_pv(G - 1, j - 1 == 0, units_with_blocks)) {
+                        ok = false;
+                        break;
+                    }
                 }
                 umma_commit(&sm.q_empty[qb]);
                 if (!ok) break;
@@ -304,6 +366,9 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
             const int u = blockIdx.x + ui * gridDim.x;
             if (u >= p.num_units) break;
             const Unit x = unit_of(p, u);
+            const int qb = ui & 1;
+            if (!mbar_wait(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err)) break;
+            const int* uidx = sm.idx[qb];
             // l_part: sums of the bf16 probabilities fed to the PV product (normalises O);
             // l_lse: the same sums before rounding (for the log-sum-exp output)
             float m_ref[kH], l_part[kH], l_lse[kH];
@@ -315,7 +380,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
                 const uint32_t ph = (G >> 1) & 1;
                 // validity of this thread's key slot (M=64 layout: lanes 0..15 of each quadrant)
                 const int r = quad * 16 + lane;
-                const bool valid = lane < 16 && resolve_row(p, x, x.e0 + j * kBK + r, false) >= 0;
+                const bool valid = lane < 16 && resolve_row(p, x, uidx, x.e0 + j * kBK + r, false) >= 0;
                 if (!mbar_wait(&sm.s_full[s], ph, abort, p.err)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t sr[16];
@@ -325,35 +390,52 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
 #pragma unroll
                 for (int h = 0; h < kH; ++h)
                     xs[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
-                // block max per head: 16-lane reduction, then across the 4 warps
+                // block max per head: one redux per head over the warp, then across the 4
+                // warps through shared memory (vector stores / loads, no branches)
+                float wmax[kH];
 #pragma unroll
-                for (int h = 0; h < kH; ++h) {
-                    float mh = xs[h];
-                    mh = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 8));
-                    mh = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 4));
-                    mh = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 2));
-                    mh = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 1));
-                    if (lane == 0) sm.red[s][quad][h] = mh;
+                for (int h = 0; h < kH; ++h)
+                    wmax[h] = order_key_to_float(
+                        __reduce_max_sync(0xffffffffu, float_order_key(xs[h])));
+                if (lane == 0) {
+                    float4* dst = reinterpret_cast<float4*>(sm.red[s][quad]);
+#pragma unroll
+                    for (int h4 = 0; h4 < kH / 4; ++h4)
+                        dst[h4] = make_float4(wmax[4 * h4], wmax[4 * h4 + 1], wmax[4 * h4 + 2],
+                                              wmax[4 * h4 + 3]);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.red_bar[s]);
                 if (!mbar_wait(&sm.red_bar[s], ph, abort, p.err)) { ok = false; break; }
+                float mb[kH];
+#pragma unroll
+                for (int h4 = 0; h4 < kH / 4; ++h4) {
+                    const float4 a = reinterpret_cast<const float4*>(sm.red[s][0])[h4];
+                    const float4 b = reinterpret_cast<const float4*>(sm.red[s][1])[h4];
+                    const float4 c = reinterpret_cast<const float4*>(sm.red[s][2])[h4];
+                    const float4 d = reinterpret_cast<const float4*>(sm.red[s][3])[h4];
+                    mb[4 * h4 + 0] = fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, d.x));
+                    mb[4 * h4 + 1] = fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, d.y));
+                    mb[4 * h4 + 2] = fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, d.z));
+                    mb[4 * h4 + 3] = fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, d.w));
+                }
+                // lazy reference: a head's reference moves only when its block max exceeds
+                // it by more than 2^8 (or when it had no valid key yet); the decision is the
+                // same in every thread because all read the same maxima
                 bool rescale = false;
-                float alpha[kH];
+                float new_ref[kH];
 #pragma unroll
                 for (int h = 0; h < kH; ++h) {
-                    const float mb = fmaxf(fmaxf(sm.red[s][0][h], sm.red[s][1][h]),
-                                           fmaxf(sm.red[s][2][h], sm.red[s][3][h]));
-                    alpha[h] = 1.f;
-                    if (m_ref[h] == -INFINITY) {
-                        m_ref[h] = mb;  // nothing accumulated yet for this head
-                    } else if (mb > m_ref[h] + kRescaleThreshold) {
-                        alpha[h] = exp2f(m_ref[h] - mb);
-                        m_ref[h] = mb;
-                        rescale = true;
-                    }
+                    const bool empty = m_ref[h] == -INFINITY;
+                    const bool grow = !empty && mb[h] > m_ref[h] + kRescaleThreshold;
+                    rescale |= grow;
+                    new_ref[h] = (empty || grow) ? mb[h] : m_ref[h];
                 }
                 if (rescale) {
+                    float alpha[kH];
+#pragma unroll
+                    for (int h = 0; h < kH; ++h)
+                        alpha[h] = m_ref[h] == -INFINITY ? 1.f : exp2f(m_ref[h] - new_ref[h]);
                     // all earlier PV products must have landed before O is scaled in place
                     const uint32_t Gp = G - 1;
                     if (!mbar_wait(&sm.pv_done[Gp & 1], (Gp >> 1) & 1, abort, p.err)) { ok = false; break; }
@@ -372,13 +454,17 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
 #pragma unroll
                     for (int h = 0; h < kH; ++h) { l_part[h] *= alpha[h]; l_lse[h] *= alpha[h]; }
                 }
+#pragma unroll
+                for (int h = 0; h < kH; ++h) m_ref[h] = new_ref[h];
                 // P buffer s is free once the PV product of block G-2 has completed
                 if (!mbar_wait(&sm.pv_done[s], ph ^ 1, abort, p.err)) { ok = false; break; }
                 if (lane < 16) {
                     uint8_t* pb = sm.p[s];
 #pragma unroll
                     for (int h = 0; h < kH; ++h) {
-                        const float pv = valid ? exp2f(xs[h] - m_ref[h]) : 0.f;
+                        // invalid keys carry xs = -inf, so exp2 gives exactly 0
+                        const float ref = m_ref[h] == -INFINITY ? 0.f : m_ref[h];
+                        const float pv = exp2f(xs[h] - ref);
                         const __nv_bfloat16 b = __float2bfloat16_rn(pv);
                         l_part[h] += __bfloat162float(b);
                         l_lse[h] += pv;
@@ -461,6 +547,8 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const MlaParams
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.o_free);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.q_empty[qb]);  // done with this unit's indices
         }
     }
 
