@@ -169,6 +169,32 @@ dsa_status dsa_sparse_mla_fwd(int dtype, int mode, int num_q, int H, int num_kv_
 size_t dsa_sparse_mla_workspace_size(int mode, int num_q, int H, int D_v, int k_sel);
 
 /*
+ * dsa_sparse_mla_decode_noalloc -- the decode path of dsa_sparse_mla_fwd (bf16 absorbed
+ * MLA, mode DSA_DECODE, same arguments and results) for callers that cannot allocate
+ * device memory where they decode, e.g. inside a fixed-size memory pool or an
+ * allocation-free serving loop.  The paper has no counterpart: this is a deployment
+ * variant of the same computation.
+ *
+ * Instead of a caller workspace, the per-split partial results live in a 16 MiB device
+ * array that belongs to the library; every GPU that loads the library holds it until
+ * the process exits.  The call allocates nothing (no cudaMalloc, cudaFree or allocating
+ * library routine).  Limits: num_q <= 511 sequences (fewer splits per sequence are used
+ * when many sequences share the array); otherwise DSA_ERR_UNSUPPORTED, before anything is
+ * launched.  The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream capture.
+ * All calls share the one array: calls that overlap on the GPU (other streams, other host
+ * threads) race and must be serialised by the caller.  Each call overwrites the parts of
+ * the array it uses, so nothing has to be cleared between calls.  Errors: as for
+ * dsa_sparse_mla_fwd (dsa_last_error() is not set by this call).
+ */
+dsa_status dsa_sparse_mla_decode_noalloc(int num_q, int H, int D_qk, int D_v, float scale,
+                                         const void* q, const void* kv, long long kv_rows,
+                                         const int* page_table, int max_pages, int page_size,
+                                         const int* seq_lens, const int* idx, int k_sel,
+                                         long long ld_idx, void* out, float* lse,
+                                         dsa_stream_t stream);
+
+/*
  * dsa_layer_stack -- IndexCache over an F/S layer pattern (vLLM IndexCache docs, "How It
  * Works"; DSV2-Lite-IndexCache card: "FSS" x 9).  Prefill, bf16 absorbed MLA.
  *

@@ -35,6 +35,8 @@ SYMBOLS = [
     ("dsa_sparse_mla_fwd", _I, [_I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _LL, _P, _I, _I, _P,
                                 _P, _I, _LL, _P, _P, _P, _SZ, _P]),
     ("dsa_sparse_mla_workspace_size", _SZ, [_I, _I, _I, _I, _I]),
+    ("dsa_sparse_mla_decode_noalloc", _I, [_I, _I, _I, _I, _F, _P, _P, _LL, _P, _I, _I, _P, _P, _I,
+                                           _LL, _P, _P, _P]),
     ("dsa_layer_stack", _I, [ctypes.c_char_p, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P,
                              _P, _P, _P, _P, _P, _SZ, _P]),
     ("dsa_layer_stack_workspace_size", _SZ, [_I, _I]),
