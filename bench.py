@@ -38,6 +38,8 @@ def parse_args(argv=None):
     ap.add_argument("--topk", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--window-rows", type=int, default=0,
+                    help="query rows per indexer/top-k window (0 = the library default)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args(argv)
@@ -219,7 +221,7 @@ def run_native(args, rank, world, local_rank):
     names = ("q_idx", "k_idx", "w", "q", "kv")
     x = {n: host[n].to(dev) for n in names}
     ld = (T + 3) // 4 * 4
-    ws_bytes = dsa.layer_stack_workspace_size(T)
+    ws_bytes = dsa.layer_stack_workspace_size(T, args.window_rows)
     rw = max(16, ws_bytes // (4 * ld))
     rw = min(T, rw // 16 * 16 if rw > 16 else rw)
     scores = torch.empty((rw, ld), dtype=torch.float32, device=dev)
