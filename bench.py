@@ -38,6 +38,9 @@ def parse_args(argv=None):
     ap.add_argument("--topk", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workload", choices=["prefill", "decode", "stack"], default="prefill",
+                    help="prefill: the T=65536 headline; decode: 64 sequences x 32768 paged "
+                         "tokens; stack: the 27-layer FSS x 9 IndexCache stack at T=16384")
     ap.add_argument("--window-rows", type=int, default=0,
                     help="query rows per indexer/top-k window (0 = the library default)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -324,7 +327,7 @@ def run_native(args, rank, world, local_rank):
                 "index_phase_ms": idx_ms}
         # dominant kernel
         if mla_ms >= indexer_ms:
-            dom, flop, fname = "sparse_mla_tc_kernel", work["mla_flop"], "mla_tc.cu"
+            dom, flop, fname = "sparse_mla_mma_kernel", work["mla_flop"], "mla_mma.cu"
             dom_ms = mla_ms
         else:
             dom, flop, fname = "indexer_tc_kernel", work["indexer_flop"], "indexer_tc.cu"
@@ -379,6 +382,106 @@ def run_native(args, rank, world, local_rank):
     return result
 
 
+def _timed(step, steps, warmup, stream):
+    """Device time of `steps` calls of step() after `warmup` calls (CUDA events)."""
+    import torch
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def run_decode(args, local_rank):
+    """Batched sparse-MLA decode step: 64 sequences of 32768 cached tokens in 64-token
+    pages; decode indexer over all cached keys + top-2048 + sparse MLA (split-k)."""
+    import torch
+    import sparse_attention_17_b200 as dsa
+    from sparse_attention_17_b200 import inputs as G
+    torch.cuda.set_device(local_rank)
+    B, L, k = 64, 32768, args.topk
+    host = G.mla_decode(B=B, L=L, k=k)
+    x = {n: host[n].cuda() for n in ("q_idx", "w", "k_idx_pool", "q", "kv_pool", "page_table",
+                                      "seq_lens")}
+    scores = torch.empty((B, L), dtype=torch.float32, device="cuda")
+    idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    out = torch.empty((B, 16, 512), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(dsa.sparse_mla_workspace_size(B, k, decode=True) // 4 + 4, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def indexer():
+        dsa.indexer_scores(x["q_idx"], x["k_idx_pool"], x["w"], scores,
+                           page_table=x["page_table"], seq_lens=x["seq_lens"])
+
+    def topk():
+        dsa.topk_select(scores, k, idx, row_len=x["seq_lens"], max_len=L)
+
+    def mla():
+        dsa.sparse_mla_fwd(x["q"], x["kv_pool"], idx, out, G.SCALE_MLA, page_table=x["page_table"],
+                           seq_lens=x["seq_lens"], workspace=ws)
+
+    def step():
+        indexer(); topk(); mla()
+
+    ms = _timed(step, args.steps, args.warmup, stream)
+    t_idx = _timed(indexer, args.steps, 1, stream)
+    t_topk = _timed(topk, args.steps, 1, stream)
+    t_mla = _timed(mla, args.steps, 1, stream)
+    assert dsa.check_device_errors() == 0
+    peaks, src = load_peaks()
+    gather = B * k * 1152
+    kidx = B * L * 64 * 2
+    return {"metric": "DSA decode sequences/sec (64 x 32768 paged, top-2048)", "value":
+            round(B / (ms / 1e3), 1), "unit": "sequences/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "dsa_decode_B64_L32768_top2048", "page_size": 64},
+            "kernels": {"indexer_ms": round(t_idx, 4), "topk_ms": round(t_topk, 4),
+                        "sparse_mla_decode_ms": round(t_mla, 4)},
+            "derived": {"indexer_key_read_gbs": round(kidx / (t_idx / 1e3) / 1e9, 1),
+                        "mla_gather_gbs": round(gather / (t_mla / 1e3) / 1e9, 1),
+                        "mla_gather_frac_of_hbm": round(gather / (t_mla / 1e3) / 1e9
+                                                        / peaks["hbm_gbs"], 4),
+                        "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": src}}
+
+
+def run_stack(args, local_rank):
+    """The IndexCache stack: 27 layers "FSS" x 9 at T=16384, top-2048, through
+    dsa_layer_stack (9 indexer + top-k passes, 27 sparse MLA passes)."""
+    import torch
+    import sparse_attention_17_b200 as dsa
+    from sparse_attention_17_b200 import inputs as G
+    torch.cuda.set_device(local_rank)
+    T, k, pattern = 16384, args.topk, "FSS" * 9
+    st = G.layer_stack(T=T, pattern=pattern, k=k)
+    layers = [{n: v.cuda() for n, v in L.items()} for L in st["layers"]]
+    outs = [torch.empty((T, 16, 512), dtype=torch.bfloat16, device="cuda") for _ in layers]
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    ws = torch.empty(dsa.layer_stack_workspace_size(T, args.window_rows) // 4, device="cuda")
+    stream = torch.cuda.current_stream()
+    dsa.reset_launch_counts()
+    ms = _timed(lambda: dsa.layer_stack(pattern, layers, idx, ws, k, G.SCALE_MLA, outs),
+                args.steps, args.warmup, stream)
+    n_calls = args.steps + args.warmup
+    launches = {kk: dsa.launch_count(i) // n_calls for i, kk in
+                enumerate(["indexer", "topk", "attention", "combine"])}
+    assert dsa.check_device_errors() == 0
+    work = algorithmic_work(T, k)
+    return {"metric": "IndexCache layer-stack tokens/sec (27 layers FSS x 9, T=16384, top-2048)",
+            "value": round(T / (ms / 1e3), 1), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "dsa_indexcache_stack_T16384_FSSx9"},
+            "launches_per_call": launches,
+            "derived": {"tflop_per_call": round((9 * work["indexer_flop"] + 27 * work["mla_flop"])
+                                                / 1e12, 2)}}
+
+
 def run_reference(args, rank, world):
     """The CPU oracle, as it stands, on bounded samples of the same workload."""
     if rank != 0:
@@ -429,7 +532,12 @@ def main(argv=None):
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
     try:
-        res = run_native(args, rank, world, local_rank)
+        if args.workload == "decode":
+            res = run_decode(args, local_rank) if rank == 0 else None
+        elif args.workload == "stack":
+            res = run_stack(args, local_rank) if rank == 0 else None
+        else:
+            res = run_native(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -108,7 +108,6 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
 }
 
 size_t topk_smem_bytes(int max_len);
-size_t mla_smem_bytes();
 
 // Validation shared by the calls.
 dsa_status check_stream_device(DevCtx* ctx) {
@@ -280,7 +279,7 @@ dsa_status dsa_sparse_mla_fwd(int dtype, int mode, int num_q, int H, int num_kv_
                     "bf16 MLA path: k_sel <= 2048 and k_sel, ld_idx multiples of 4");
     if (mode == DSA_PREFILL) {
         if (page_table || seq_lens) return fail(DSA_ERR_INVALID_ARG, "prefill takes no pages");
-        e = launch_sparse_mla_bf16(static_cast<const __nv_bfloat16*>(q),
+        e = launch_sparse_mla_mma(static_cast<const __nv_bfloat16*>(q),
                                    static_cast<const __nv_bfloat16*>(kv), kv_rows, nullptr, 0, 0,
                                    nullptr, idx, k_sel, ld_idx, num_q, scale, 1,
                                    static_cast<__nv_bfloat16*>(out), lse, nullptr, nullptr, cs, ctx);
@@ -297,7 +296,7 @@ dsa_status dsa_sparse_mla_fwd(int dtype, int mode, int num_q, int H, int num_kv_
     if (!aligned16(workspace)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
     float* o_part = static_cast<float*>(workspace);
     float* lse_part = o_part + (size_t)num_q * splits * H * D_v;
-    e = launch_sparse_mla_bf16(static_cast<const __nv_bfloat16*>(q),
+    e = launch_sparse_mla_mma(static_cast<const __nv_bfloat16*>(q),
                                static_cast<const __nv_bfloat16*>(kv), kv_rows, page_table,
                                max_pages, page_size, seq_lens, idx, k_sel, ld_idx, num_q, scale,
                                splits, nullptr, nullptr, o_part, lse_part, cs, ctx);
@@ -312,9 +311,10 @@ size_t dsa_layer_stack_workspace_size(int T, int rows_window) {
     const long long ld = ((long long)T + 3) / 4 * 4;
     long long rw = rows_window;
     if (rw <= 0) {
-        // default: about 64 MB of scores per window (stays mostly in the 126 MB L2),
-        // at least 128 rows
-        rw = (64ll << 20) / (ld * 4);
+        // default: about 512 MB of scores per window.  Wider windows give the indexer and
+        // top-k launches enough rows to fill the GPU; at T = 65536 this is 2048 rows
+        // (the index phase measured 22.8 ms with 256-row windows, 15.9 ms with 2048).
+        rw = (512ll << 20) / (ld * 4);
         if (rw < 128) rw = 128;
     }
     if (rw > T) rw = T;

@@ -1,7 +1,7 @@
 // simt_f32.cu -- fp32 kernels for the small DSA layer of the DSA ablation model card
 // (lightning indexer with 2 heads x dim 16, top-512, 4 attention heads of dim 32, context
 // 3072).  The work is about 1 GFLOP in total, so these are plain SIMT kernels; the bf16
-// paths for the 576-dim MLA layers run on tcgen05 (indexer_tc.cu, mla_tc.cu).
+// paths for the 576-dim MLA layers are indexer_tc.cu (tcgen05) and mla_mma.cu.
 #include "dsa_common.cuh"
 #include "launch.h"
 

@@ -132,7 +132,7 @@ def test_workspace_sizes(lib):
     assert lib.dsa_sparse_mla_workspace_size(0, 100, 16, 512, 2048) == 0
     ws = lib.dsa_sparse_mla_workspace_size(1, 64, 16, 512, 2048)
     assert ws > 0 and ws % (64 * 16 * 513 * 4) == 0
-    assert lib.dsa_layer_stack_workspace_size(65536, 0) == 64 << 20
+    assert lib.dsa_layer_stack_workspace_size(65536, 0) == 512 << 20
     assert lib.dsa_layer_stack_workspace_size(1000, 0) == 1000 * 1000 * 4
     assert lib.dsa_layer_stack_workspace_size(100, 16) == 16 * 100 * 4
 
