@@ -128,7 +128,8 @@ dsa_status dsa_indexer_scores(int dtype, int mode, const void* q_idx, const void
  * scores; among equal scores the lower index wins (-0.0 and +0.0 are equal).  If n_r <= k
  * all n_r keys are selected.  idx[r * ld_idx + i], i < k, receives the selected key
  * positions in ascending order followed by -1 padding.  Scores must not be NaN.
- * Limits: 1 <= k <= 4096, max_len <= 262144, ld_idx >= k.
+ * Limits: 1 <= k <= 4096, max_len <= 262144, ld_idx >= k, ld_scores a multiple of 4
+ * (rows start on 16-byte boundaries); scores, idx and row_len 16-byte aligned.
  */
 dsa_status dsa_topk_select(const float* scores, long long ld_scores, int rows, int q_begin,
                            const int* row_len, int max_len, int k, int* idx,

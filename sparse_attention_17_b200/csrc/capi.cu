@@ -217,6 +217,8 @@ dsa_status dsa_topk_select(const float* scores, long long ld_scores, int rows, i
     if (max_len < 1 || max_len > 262144)
         return fail(DSA_ERR_UNSUPPORTED, "max_len must be in [1, 262144]");
     if (max_len > ld_scores) return fail(DSA_ERR_INVALID_ARG, "max_len > ld_scores");
+    if (ld_scores & 3)
+        return fail(DSA_ERR_INVALID_ARG, "ld_scores must be a multiple of 4 (16-byte rows)");
     if (!row_len && (long long)q_begin + rows > max_len)
         return fail(DSA_ERR_INVALID_ARG, "causal rows need max_len >= q_begin + rows");
     if (rows == 0) return DSA_OK;

@@ -109,6 +109,8 @@ def test_topk_rejects(lib):
     assert lib.dsa_topk_select(16, 32, 4, 0, None, 64, 8, 16, 8, None) == _lib.DSA_ERR_INVALID_ARG
     # causal rows beyond max_len
     assert lib.dsa_topk_select(16, 64, 70, 0, None, 64, 8, 16, 8, None) == _lib.DSA_ERR_INVALID_ARG
+    # score rows must start on 16-byte boundaries (ld a multiple of 4)
+    assert lib.dsa_topk_select(16, 66, 4, 0, None, 64, 8, 16, 8, None) == _lib.DSA_ERR_INVALID_ARG
     assert lib.dsa_topk_select(16, 64, 0, 0, None, 64, 8, 16, 8, None) == _lib.DSA_OK
 
 
