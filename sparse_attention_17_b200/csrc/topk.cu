@@ -5,17 +5,20 @@
 // n <= k every key is selected.  Output: the selected key positions in ascending order,
 // then -1 padding.
 //
-// One CTA of 512 threads per row.  Scores map to order-preserving uint32 keys.
+// One CTA of 512 threads per row.  Scores map to order-preserving uint32 keys.  Each warp
+// owns a 512-entry slice of the shared candidate buffer, so candidates are appended with
+// a ballot and a popcount and no shared atomics.
 // Fast path (one read of the row):
-//   sample  every 16th 32-key chunk of the row goes to shared memory; an exact radix
-//           select there picks a provisional threshold tau0 a few standard deviations
-//           below the sample's k-th-largest-equivalent rank (rows of at most 8192 keys
-//           skip this: tau0 = the smallest key);
-//   gather  one vectorised pass appends every key >= tau0 to a shared candidate list
-//           (warp ballots, one shared atomic per warp);
+//   sample  every 16th 32-key chunk of the row (at most 256 chunks, all loads in flight
+//           at once) goes to the slices; a two-round (12 + 12 bit) radix select there
+//           gives a provisional threshold tau0 below the sample rank that corresponds to
+//           k plus a few standard deviations (rows of at most 8192 keys skip this:
+//           tau0 = the smallest key);
+//   gather  one pass with four 16-byte loads per thread in flight appends every key
+//           >= tau0 to the warp's slice (128-key chunks dealt round-robin to the warps);
 //   select  radix select (12 + 12 + 8 bits) among the candidates gives the k-th largest
 //           key tau; candidates above tau are selected, those equal to tau are ties.
-// If the candidates number fewer than k or more than the buffer holds, the row is redone
+// If the candidates number fewer than k or more than a slice holds, the row is redone
 // exactly from global memory (histogram passes over the whole row).  Finally the first
 // `need` ties in index order are kept and a bitmap of the selection is compacted in index
 // order, which yields ascending indices without sorting.
@@ -31,18 +34,22 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 4096;
 constexpr int kCandCap = 8192;
 constexpr int kStride = kWarps * 32;  // elements covered by all warps per iteration
+constexpr int kSlice = kCandCap / kWarps;  // candidate entries owned by one warp
+constexpr int kUnroll = 4;                 // 16-byte loads in flight per thread
 
 struct TopkScratch {
     uint32_t hist[kBins];
     uint32_t cand_key[kCandCap];
     int cand_idx[kCandCap];
     uint32_t scan[kWarps];
+    uint32_t wcount[kWarps];  // candidates appended by each warp (may exceed kSlice)
     uint32_t cand_count;
     uint32_t found_bin;
     uint32_t found_above;
 };
 
 constexpr int kSampleChunks = kCandCap / 32;  // at most 256 sampled 32-key chunks
+constexpr int kSampleChunksPerWarp = kSampleChunks / kWarps;  // 16 chunks = one slice
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
@@ -115,14 +122,19 @@ __device__ __forceinline__ void zero_hist(TopkScratch& sh, int nbins) {
     for (int i = threadIdx.x; i < nbins; i += kThreads) sh.hist[i] = 0u;
 }
 
-// Exact radix select of the `need`-th largest of keys[0..cnt) (shared memory): returns the
-// key value tau; *need_out = how many keys equal to tau belong to the top `need`.
-__device__ uint32_t smem_radix_select(TopkScratch& sh, const uint32_t* keys, int cnt,
-                                      uint32_t need, uint32_t* need_out) {
+// Radix select over the warps' candidate slices (warp w owns cand_key[w * kSlice ..] with
+// wcount[w] <= kSlice entries).  exact: returns the need-th largest key tau and sets
+// *need_out to how many keys equal to tau belong to the top `need` (12 + 12 + 8 bits).
+// !exact: stops after 24 bits and returns the lower edge of the 24-bit bin holding the
+// need-th largest key, a lower bound of it.
+__device__ uint32_t slice_radix_select(TopkScratch& sh, uint32_t need, bool exact,
+                                       uint32_t* need_out) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t* keys = sh.cand_key + warp * kSlice;
+    const int cnt = (int)sh.wcount[warp];
     zero_hist(sh, kBins);
     __syncthreads();
-    for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
+    for (int c0 = 0; c0 < cnt; c0 += 32) {
         const int c = c0 + lane;
         hist_add(sh.hist, c < cnt ? keys[c] >> 20 : 0u, c < cnt);
     }
@@ -132,7 +144,7 @@ __device__ uint32_t smem_radix_select(TopkScratch& sh, const uint32_t* keys, int
     need -= sh.found_above;
     zero_hist(sh, kBins);
     __syncthreads();
-    for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
+    for (int c0 = 0; c0 < cnt; c0 += 32) {
         const int c = c0 + lane;
         const uint32_t key = c < cnt ? keys[c] : 0u;
         hist_add(sh.hist, (key >> 8) & 0xFFFu, c < cnt && (key >> 20) == b1);
@@ -141,9 +153,14 @@ __device__ uint32_t smem_radix_select(TopkScratch& sh, const uint32_t* keys, int
     find_bin(sh, kBins, need);
     const uint32_t pre = (b1 << 12) | sh.found_bin;
     need -= sh.found_above;
+    if (!exact) {
+        *need_out = need;
+        __syncthreads();
+        return pre << 8;
+    }
     zero_hist(sh, 256);
     __syncthreads();
-    for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
+    for (int c0 = 0; c0 < cnt; c0 += 32) {
         const int c = c0 + lane;
         const uint32_t key = c < cnt ? keys[c] : 0u;
         hist_add(sh.hist, key & 0xFFu, c < cnt && (key >> 8) == pre);
@@ -315,73 +332,98 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
     const float* row = scores + (long long)r * ld;
     const int nwords = (n + 31) >> 5;
     for (int i = threadIdx.x; i < nwords; i += kThreads) tie[i] = 0u;
-    if (threadIdx.x == 0) sh.cand_count = 0u;
     __syncthreads();
 
     // ---- provisional threshold from a sample of the row ----
     uint32_t tau0 = 0u;
+    const uint32_t slice0 = (uint32_t)warp * kSlice;
     if (n > kCandCap) {
         const int nchunks = (n + 31) >> 5;
         const int stride = max(16, (nchunks + kSampleChunks - 1) / kSampleChunks);
-        const int nsamp = (nchunks + stride - 1) / stride;  // sampled chunks
-        uint32_t valid = 0;
-        for (int j = warp; j < nsamp; j += kWarps) {
+        const int nsamp = (nchunks + stride - 1) / stride;  // sampled chunks, <= 256
+        float xs[kSampleChunksPerWarp];
+#pragma unroll
+        for (int i = 0; i < kSampleChunksPerWarp; ++i) {
+            const int j = warp + i * kWarps;
             const int sidx = j * stride * 32 + lane;
-            const bool in = sidx < n;
-            sh.cand_key[j * 32 + lane] = in ? float_order_key(__ldg(row + sidx)) : 0u;
-            valid += __popc(__ballot_sync(0xffffffffu, in));
+            xs[i] = (j < nsamp && sidx < n) ? __ldg(row + sidx) : 0.f;
         }
-        if (lane == 0) atomicAdd(&sh.cand_count, valid);
+        uint32_t cnt = 0;
+#pragma unroll
+        for (int i = 0; i < kSampleChunksPerWarp; ++i) {
+            const int j = warp + i * kWarps;
+            const int sidx = j * stride * 32 + lane;
+            const bool in = j < nsamp && sidx < n;
+            const unsigned m = __ballot_sync(0xffffffffu, in);
+            if (in) sh.cand_key[slice0 + cnt + __popc(m & lanemask_lt())] = float_order_key(xs[i]);
+            cnt += __popc(m);
+        }
+        if (lane == 0) sh.wcount[warp] = cnt;
         __syncthreads();
-        const uint32_t m = sh.cand_count;
+        uint32_t m = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) m += sh.wcount[w];
         // rank in the sample whose key should leave >= k keys of the row above it
         const float expect = (float)k * (float)m / (float)n;
         uint32_t rank = (uint32_t)ceilf(expect + 3.f * sqrtf(expect)) + 2u;
         if (rank > m) rank = m;
         uint32_t dummy;
-        tau0 = smem_radix_select(sh, sh.cand_key, nsamp * 32, rank, &dummy);
-        if (threadIdx.x == 0) sh.cand_count = 0u;
-        __syncthreads();
+        tau0 = slice_radix_select(sh, rank, false, &dummy);
     }
 
-    // ---- one pass: every key >= tau0 becomes a candidate ----
-    for (int base = warp * 128; base < n; base += kWarps * 128) {
-        const int s0 = base + 4 * lane;
-        float x[4];
-        if (s0 + 3 < n) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(row + s0));
-            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-        } else {
+    // ---- one pass: every key >= tau0 becomes a candidate in this warp's slice ----
+    uint32_t cnt = 0;
+    for (int base = warp * 128; base < n; base += kWarps * 128 * kUnroll) {
+        float4 v[kUnroll];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) x[u] = s0 + u < n ? __ldg(row + s0 + u) : 0.f;
+        for (int u = 0; u < kUnroll; ++u) {
+            const int s0 = base + u * kWarps * 128 + 4 * lane;
+            if (s0 + 3 < n) {
+                v[u] = __ldg(reinterpret_cast<const float4*>(row + s0));
+            } else {
+                v[u].x = s0 < n ? __ldg(row + s0) : 0.f;
+                v[u].y = s0 + 1 < n ? __ldg(row + s0 + 1) : 0.f;
+                v[u].z = s0 + 2 < n ? __ldg(row + s0 + 2) : 0.f;
+                v[u].w = 0.f;
+            }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const uint32_t key = float_order_key(x[u]);
-            const bool take = s0 + u < n && key >= tau0;
-            const unsigned m = __ballot_sync(0xffffffffu, take);
-            if (m) {
-                uint32_t pos0 = 0;
-                if (lane == 0) pos0 = atomicAdd(&sh.cand_count, (uint32_t)__popc(m));
-                pos0 = __shfl_sync(0xffffffffu, pos0, 0);
-                const uint32_t p = pos0 + __popc(m & lanemask_lt());
-                if (take && p < (uint32_t)kCandCap) {
-                    sh.cand_key[p] = key;
-                    sh.cand_idx[p] = s0 + u;
+        for (int u = 0; u < kUnroll; ++u) {
+            const int s0 = base + u * kWarps * 128 + 4 * lane;
+            const float xv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t key = float_order_key(xv[e]);
+                const bool take = s0 + e < n && key >= tau0;
+                const unsigned m = __ballot_sync(0xffffffffu, take);
+                if (take) {
+                    const uint32_t p = cnt + __popc(m & lanemask_lt());
+                    if (p < (uint32_t)kSlice) {
+                        sh.cand_key[slice0 + p] = key;
+                        sh.cand_idx[slice0 + p] = s0 + e;
+                    }
                 }
+                cnt += __popc(m);
             }
         }
     }
     for (int i = threadIdx.x; i < nwords; i += kThreads) sel[i] = 0u;
+    __syncthreads();  // everyone is past the sample select before wcount is rewritten
+    if (lane == 0) sh.wcount[warp] = cnt;
     __syncthreads();
-    const uint32_t ncand = sh.cand_count;
-    __syncthreads();  // everyone has read the count before it can be reused
+    uint32_t ncand = 0;
+    bool overflow = false;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        ncand += sh.wcount[w];
+        overflow |= sh.wcount[w] > (uint32_t)kSlice;
+    }
     uint32_t need;
-    if (ncand >= (uint32_t)k && ncand <= (uint32_t)kCandCap) {
-        const uint32_t tau = smem_radix_select(sh, sh.cand_key, (int)ncand, (uint32_t)k, &need);
-        for (int c = threadIdx.x; c < (int)ncand; c += kThreads) {
-            const uint32_t key = sh.cand_key[c];
-            const int sidx = sh.cand_idx[c];
+    if (!overflow && ncand >= (uint32_t)k) {
+        const uint32_t tau = slice_radix_select(sh, (uint32_t)k, true, &need);
+        for (int c = lane; c < (int)cnt; c += 32) {
+            const uint32_t key = sh.cand_key[slice0 + c];
+            const int sidx = sh.cand_idx[slice0 + c];
             if (key > tau) atomicOr(&sel[sidx >> 5], 1u << (sidx & 31));
             else if (key == tau) atomicOr(&tie[sidx >> 5], 1u << (sidx & 31));
         }

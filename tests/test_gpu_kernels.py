@@ -259,3 +259,27 @@ def test_topk_sample_miss_falls_back_to_exact():
     sc[1, ::512] = 50.0  # sampled chunk heads are huge: threshold too high, too few candidates
     idx, ref = _topk_case(sc, [S, S], k, row_len=True)
     check_indices_exact(idx, ref, "sample miss")
+
+
+def test_topk_one_warp_region_overflows_to_exact():
+    """Every large score sits in 128-key chunks that one warp of the candidate pass reads
+    (chunk index = 3 mod 16), and the threshold sample never reads those chunks: that
+    warp's candidate slice overflows and the row must be redone exactly."""
+    S, k = 65536, 2048
+    r = np.random.default_rng(11)
+    sc = r.normal(size=(2, S))
+    hot = (np.arange(S) // 128) % 16 == 3
+    sc[0, hot] = r.normal(10, 1, hot.sum())
+    sc[1, hot[:S]] = np.where(r.random(hot.sum()) < 0.2, 4.0, sc[1, hot])
+    idx, ref = _topk_case(sc, [S, S], k, row_len=True)
+    check_indices_exact(idx, ref, "one-warp overflow")
+
+
+@pytest.mark.parametrize("n_valid", [[8192, 8193, 8191, 12345, 2049, 65536, 16385, 4097]])
+def test_topk_lengths_around_sample_switch(n_valid):
+    """Rows of at most 8192 keys skip the threshold sample; longer ones use it."""
+    S, k = 65536, 2048
+    r = np.random.default_rng(12)
+    sc = r.normal(size=(len(n_valid), S)).astype(np.float32).astype(np.float64)
+    idx, ref = _topk_case(sc, n_valid, k, row_len=True)
+    check_indices_exact(idx, ref, "sample switch")
