@@ -11,10 +11,13 @@
 // With keys on lanes, the ReLU + head-weight reduction of a score is a sum over 16
 // consecutive TMEM columns that stay inside one thread -- no shuffles.
 //
-// Warp roles (384 threads): warp 0 issues TMA loads (query block once per unit, key tiles
+// Warp roles (640 threads): warp 0 issues TMA loads (query block once per unit, key tiles
 // through a ring of smem stages), warp 1 issues UMMAs into a double-buffered TMEM
-// accumulator (2 x 256 columns), warp 2 owns the TMEM allocation, warps 4..11 drain the
-// accumulator: tcgen05.ld, ReLU, weight, reduce, causal mask, coalesced fp32 stores.
+// accumulator (2 x 256 columns), warp 2 owns the TMEM allocation, warps 4..19 drain the
+// accumulator: tcgen05.ld, ReLU, weight, reduce, causal mask, coalesced fp32 stores.  The
+// drain is the longest stage per tile (16 max + 16 multiply-adds per score), so it gets
+// four warps per TMEM lane quadrant, each on a quarter of the tile's queries, and the head
+// weights are applied with packed fp32x2 FMAs.
 //
 // Work units are (query block, chunk of at most 32 key tiles): prefill blocks hold 16
 // queries and their causal key range grows with the query position, so the range is cut
@@ -32,9 +35,9 @@ constexpr int kHI = 16;
 constexpr int kDI = 64;
 constexpr int kBM = 128;           // keys per tile (UMMA M)
 constexpr int kStages = 6;         // key-tile ring
-constexpr int kThreads = 384;
+constexpr int kThreads = 640;
 constexpr int kEpiWarp0 = 4;       // first epilogue warp
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;      // four per TMEM lane quadrant
 constexpr uint32_t kTileBytes = kBM * 128;  // 128 keys x 64 bf16
 constexpr int kDecodeChunkTiles = 16;       // decode unit = 2048 keys
 constexpr int kPrefillChunkTiles = 32;      // prefill unit: at most 4096 keys
@@ -67,6 +70,15 @@ struct IdxParams {
     int max_pages, page_size, num_pages, max_len;
     unsigned* err;
 };
+
+// d0 += a0 * b0, d1 += a1 * b1 as one packed fp32x2 FMA (PTX fma.rn.f32x2, sm_100a): each
+// lane is rounded once, exactly like fmaf
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 pa, pb, pc;\n\t"
+        "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\tmov.b64 pc, {%0, %1};\n\t"
+        "fma.rn.f32x2 pc, pa, pb, pc;\n\tmov.b64 {%0, %1}, pc;\n\t}"
+        : "+f"(d0), "+f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
 
 // Unit visited by this CTA at step i (snake order over rounds of gridDim.x units).
 __device__ __forceinline__ int unit_at(int i) {
@@ -240,9 +252,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         // ---------------- epilogue ----------------
         const int ew = warp - kEpiWarp0;
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
-        const int half = ew >> 2;               // which half of the queries
-        constexpr int QPW = QB >= 2 ? QB / 2 : 1;  // queries per epilogue warp
-        const bool active_half = QB >= 2 || half == 0;
+        const int part = ew >> 2;               // which quarter of the queries
+        constexpr int QPW = QB >= 4 ? QB / 4 : 1;  // queries per epilogue warp
+        const bool active = QB >= 4 || part == 0;
         uint32_t it = 0;
         for (int i = 0, ui = 0;; ++i, ++ui) {
             const int u = unit_at(i);
@@ -250,7 +262,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const UnitInfo<QB, PAGED> x = unit_info<QB, PAGED>(p, u);
             const int qb = ui & 1;
             if (!mbar_wait(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err)) break;
-            const float* wbuf = sm.w[qb] + half * QPW * kHI;  // this warp's queries' weights
+            const float* wbuf = sm.w[qb] + part * QPW * kHI;  // this warp's queries' weights
             bool ok = true;
             for (int j = 0; j < x.ntiles; ++j, ++it) {
                 const int ab = it & 1;
@@ -259,27 +271,30 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 tc_fence_after();
                 const int s = (x.tile0 + j) * kBM + quad * 32 + lane;
                 const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + ab * kAccCols;
-                if (active_half) {
+                if (active) {
+                    constexpr int QW = QPW < 2 ? QPW : 2;  // queries per TMEM load round
 #pragma unroll
-                    for (int qi = 0; qi < QPW; qi += 2) {
-                        uint32_t ra[16], rb[16];
-                        const int i0 = half * QPW + qi;
-                        tmem_ld16(tbase + i0 * kHI, ra);
-                        if (QPW > 1) tmem_ld16(tbase + (i0 + 1) * kHI, rb);
+                    for (int qi = 0; qi < QPW; qi += QW) {
+                        uint32_t r[QW][16];
+                        const int i0 = part * QPW + qi;
+#pragma unroll
+                        for (int qq = 0; qq < QW; ++qq) tmem_ld16(tbase + (i0 + qq) * kHI, r[qq]);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int h2 = 0; h2 < (QPW > 1 ? 2 : 1); ++h2) {
-                            const int qidx = i0 + h2;
-                            const uint32_t* r = h2 == 0 ? ra : rb;
-                            const float4* w4 = reinterpret_cast<const float4*>(wbuf + (qidx - half * QPW) * kHI);
+                        for (int qq = 0; qq < QW; ++qq) {
+                            const int qidx = i0 + qq;
+                            const float4* w4 =
+                                reinterpret_cast<const float4*>(wbuf + (qidx - part * QPW) * kHI);
+                            // even heads accumulate in acc0, odd heads in acc1
                             float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
                             for (int h4 = 0; h4 < 4; ++h4) {
                                 const float4 wv = w4[h4];
-                                acc0 = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * h4 + 0]), 0.f), acc0);
-                                acc1 = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * h4 + 1]), 0.f), acc1);
-                                acc0 = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * h4 + 2]), 0.f), acc0);
-                                acc1 = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * h4 + 3]), 0.f), acc1);
+                                const uint32_t* rv = r[qq] + 4 * h4;
+                                ffma2(acc0, acc1, wv.x, wv.y, fmaxf(__uint_as_float(rv[0]), 0.f),
+                                      fmaxf(__uint_as_float(rv[1]), 0.f));
+                                ffma2(acc0, acc1, wv.z, wv.w, fmaxf(__uint_as_float(rv[2]), 0.f),
+                                      fmaxf(__uint_as_float(rv[3]), 0.f));
                             }
                             const float score = acc0 + acc1;
                             if constexpr (!PAGED) {
