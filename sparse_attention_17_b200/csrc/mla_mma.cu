@@ -1,5 +1,6 @@
 // mla_mma.cu -- sparse absorbed-MLA attention (prefill and paged decode) on warp-level
-// tensor-core MMAs (mma.sync m16n8k16, bf16 in, fp32 accumulate).
+// tensor-core MMAs (mma.sync m16n8k16, bf16 in, fp32 accumulate), with the selected
+// latent rows gathered by TMA bulk copies.
 //
 // For query n and head h (16 heads), over the selected keys I_n only:
 //   logit_s  = scale * q[n,h,0:576] . C[s,0:576]          C = 576-dim latent row
@@ -9,25 +10,35 @@
 //
 // Why warp MMAs here.  With 16 heads every product has a 16-wide side.  On this B200 a
 // tcgen05.mma with N <= 64 costs ~49 cycles per instruction whatever M is, so the 16-head
-// products (52 UMMAs per 64 keys) would be bound at ~40 cycles per key by instruction
-// issue, while m16n8k16 warp MMAs reach ~1,030 MAC/clk per SM -- about 17 cycles per key
-// for the same work.  The gather of the selected 1152-byte latent rows (cp.async, ~32
-// bytes/clk per SM from L2) is then the bound, as it should be for this operation.
+// products would be bound by UMMA issue, while m16n8k16 warp MMAs reach ~1,030 MAC/clk per
+// SM.  The gather of the selected 1152-byte rows (about 2 KB of latent data per query and
+// key block of 64 FLOP/B) is then the bound, as it should be for this operation.
 //
-// Per CTA (persistent; one query -- or one split of a decode sequence -- per unit):
-//   warps 8..11  gather: 16-byte cp.async copies of each selected row into a 64-row stage
-//                (rows padded to 1168 B so that ldmatrix reads are bank-conflict free);
-//                invalid / padding rows are zero-filled; completion on an mbarrier.
-//                Warp 8 lane 0 also bulk-copies the next unit's query and indices.
-//   warps 0..7   compute.  QK: warp w takes keys 16*(w%4)..+15 and K-half w/4 (18 of the
-//                36 K-steps); its half of Q stays in registers for the whole unit.  The
-//                two K-halves are summed through shared memory, the K-half-0 warps run
-//                the online softmax (exact running max, rescale of O in registers) and
-//                write P in bf16; then every warp computes PV for its 64 output dims
-//                (O stays in registers) and releases the stage.
-// Two stages keep the next block's gather in flight while a block is computed.  Decode
-// splits a sequence's selected keys over several units; their normalised partials and
-// log-sum-exps are merged by mla_combine_kernel.
+// Why this shape (measured).  With one CTA per SM, every phase of a block (gather, QK,
+// cross-warp exchanges, softmax, PV) ran back to back and the kernel reached ~5.3 TB/s of
+// gathered rows whatever the split of the work.  Here two independent CTAs share each SM,
+// so one CTA's exchanges and softmax overlap the other's MMAs, and the rows are fetched by
+// TMA bulk copies, which take no load/store-unit issue slots from the compute warps.
+//
+// Per CTA (two per SM, persistent; one query -- or one split of a decode sequence -- per
+// unit), 192 threads:
+//   warps 4, 5   gather: each lane of 16 issues one 1152-byte bulk copy (TMA) of its
+//                selected row into a 32-row stage (rows padded to 1168 B so that ldmatrix
+//                reads are bank-conflict free) and records whether the row is valid;
+//                completion is tracked by the stage's mbarrier transaction count.  Rows of
+//                invalid or padding entries are not fetched: they keep finite stale data
+//                and get probability exactly 0.  Warp 4 lane 0 also bulk-copies each
+//                unit's 16x576 query.  Selected indices are read from global memory one
+//                block ahead.
+//   warps 0..3   compute.  QK: warp w takes K-quarter w (9 of the 36 K-steps) for all 32
+//                keys of the block; its quarter of Q stays in registers for the whole
+//                unit.  Partial scores are exchanged through shared memory so that warp w
+//                sums the four quarters for keys 8w..8w+7, runs the online softmax on them
+//                (exact running max shared through shared memory) and writes P in bf16.
+//                PV: warp w owns 128 of the 512 output dims (O stays in registers).
+// Two stages per CTA keep the next block's gather in flight while a block is computed.
+// Decode splits a sequence's selected keys over several units; their normalised partials
+// and log-sum-exps are merged by mla_combine_kernel.
 #include "dsa_common.cuh"
 #include "launch.h"
 
@@ -38,32 +49,38 @@ namespace {
 constexpr int kH = 16;
 constexpr int kDqk = 576;
 constexpr int kDv = 512;
-constexpr int kBK = 64;                        // keys per block / stage
+constexpr int kComputeWarps = 4;
+constexpr int kBK = 32;                        // keys per block / stage
+constexpr int kCtasPerSm = 2;
+constexpr int kStages = 2;
+constexpr int kNT = kBK / 8;                   // 8-key n-tiles per block (one per compute warp)
+constexpr int kGatherWarps = kBK / 16;         // each gather warp copies 16 rows per stage
+constexpr int kGatherWarp0 = kComputeWarps;
+constexpr int kThreads = 32 * (kComputeWarps + kGatherWarps);
 constexpr int kRowPitch = 1168;                // bytes per staged key row (1152 + 16)
-constexpr int kStageBytes = kBK * kRowPitch;   // 74752
+constexpr int kStageBytes = kBK * kRowPitch;
 constexpr int kQPitch = 1168;                  // bytes per query head row
 constexpr int kQBytes = kH * kQPitch;          // 18688
-constexpr int kPPitch = 144;                   // bytes per P row (64 keys bf16 + 16)
-constexpr int kPBytes = kH * kPPitch;          // 2304
-constexpr int kIdxCap = 2048;
-constexpr int kComputeWarps = 8;
-constexpr int kGatherWarp0 = 8;
-constexpr int kGatherWarps = 4;
-constexpr int kThreads = 32 * (kComputeWarps + kGatherWarps);  // 384
+constexpr int kPPitch = kBK * 2 + 16;          // bytes per P row (bf16 keys + 16)
+constexpr int kPBytes = kH * kPPitch;
 constexpr int kKSteps = kDqk / 16;             // 36
-constexpr int kKHalf = kKSteps / 2;            // 18
+constexpr int kKQuarter = kKSteps / kComputeWarps;  // K-steps of the QK product per warp
+constexpr int kDvWarp = kDv / kComputeWarps;   // output dims per compute warp
+constexpr int kPVTiles = kDvWarp / 8;          // 8-dim n-tiles per compute warp
+static_assert(kNT == kComputeWarps, "each compute warp runs the softmax of one n-tile");
+static_assert(kKSteps % kComputeWarps == 0, "the K-steps split evenly over the warps");
+static_assert(kDvWarp % 16 == 0, "PV loads two n-tiles at a time");
 
 struct MmaSmem {
-    alignas(128) uint8_t stage[2][kStageBytes];
-    alignas(128) uint8_t q[2][kQBytes];
-    alignas(128) uint8_t p[2][kPBytes];
-    alignas(16) int idx[2][kIdxCap];
-    alignas(16) float spart[4][32][8];   // K-half-1 partial scores, per key group
-    alignas(16) float red[4][kH];        // per key group, per head block maxima
-    alignas(16) float alpha[kH];         // per head rescale factor of the current block
-    alignas(16) float lsum[4][kH];       // per key group row sums at the end of a unit
-    uint64_t a_full[2], a_free[2];
-    uint64_t q_full[2], q_empty[2];
+    alignas(128) uint8_t stage[kStages][kStageBytes];
+    alignas(128) uint8_t q[kQBytes];
+    alignas(128) uint8_t p[kStages][kPBytes];
+    alignas(16) int valid[kStages][kBK];     // 1: the staged row holds the key; -1: not fetched
+    alignas(16) float spart[kComputeWarps][kNT][32][4];  // [from warp][n-tile] partial scores
+    alignas(16) float red[kStages][kComputeWarps][kH];    // per warp, per head block maxima
+    alignas(16) float lsum[2][kComputeWarps][kH];         // per warp row sums at the end of a unit
+    uint64_t a_full[kStages], a_free[kStages];
+    uint64_t q_full, q_empty;
     int abort;
 };
 
@@ -105,26 +122,28 @@ __device__ __forceinline__ Unit unit_of(const Params& p, int u) {
     return x;
 }
 
-// Cache row of index entry e (-1: padding or invalid; invalid entries are reported).
-__device__ __forceinline__ long long resolve_row(const Params& p, const Unit& x, const int* uidx,
-                                                 int e, bool report) {
-    if (e >= x.e1) return -1;
-    const int s = uidx[e - x.e0];
+// Selected key of index entry e (-1 past the unit's entries).
+__device__ __forceinline__ int load_index(const Params& p, const Unit& x, int e) {
+    return e < x.e1 ? __ldg(p.idx + (long long)x.n * p.ld_idx + e) : -1;
+}
+
+// Cache row of selected key s (-1: padding or invalid; invalid keys are reported).
+__device__ __forceinline__ long long resolve_row(const Params& p, const Unit& x, int s) {
     if (s < 0) return -1;
     if (p.page_table == nullptr) {
         if (s >= p.kv_rows) {
-            if (report) atomicOr(p.err, DSA_DEVERR_INDEX_RANGE);
+            atomicOr(p.err, DSA_DEVERR_INDEX_RANGE);
             return -1;
         }
         return s;
     }
     if (s >= x.len) {
-        if (report) atomicOr(p.err, DSA_DEVERR_INDEX_RANGE);
+        atomicOr(p.err, DSA_DEVERR_INDEX_RANGE);
         return -1;
     }
     const int pg = __ldg(p.page_table + (long long)x.n * p.max_pages + s / p.page_size);
     if (pg < 0 || pg >= p.num_pages) {
-        if (report) atomicOr(p.err, DSA_DEVERR_PAGE_RANGE);
+        atomicOr(p.err, DSA_DEVERR_PAGE_RANGE);
         return -1;
     }
     return (long long)pg * p.page_size + s % p.page_size;
@@ -166,7 +185,7 @@ __device__ __forceinline__ void wait_soft(uint64_t* bar, uint32_t parity, volati
     (void)mbar_wait(bar, parity, abort, err);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 sparse_mla_mma_kernel(const Params p) {
     extern __shared__ uint8_t smem_raw[];
     MmaSmem& sm = *reinterpret_cast<MmaSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -175,17 +194,19 @@ sparse_mla_mma_kernel(const Params p) {
     volatile int* abort = &sm.abort;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&sm.a_full[i], 32 * kGatherWarps);  // one cp.async arrival per gather thread
+        for (int i = 0; i < kStages; ++i) {
+            // one expect-tx arrival per gather warp (after it has written the stage's valid
+            // flags); the phase completes when every issued row copy has landed
+            mbar_init(&sm.a_full[i], kGatherWarps);
             mbar_init(&sm.a_free[i], kComputeWarps);
-            mbar_init(&sm.q_full[i], 1);
-            mbar_init(&sm.q_empty[i], kComputeWarps + kGatherWarps);
         }
+        mbar_init(&sm.q_full, 1);
+        mbar_init(&sm.q_empty, kComputeWarps);
         sm.abort = 0;
         fence_barrier_init();
     }
-    // zero the stages once: rows of invalid keys are zero-filled by the gather anyway, and
-    // the padding columns are never read
+    // zero the stages once, so that rows never fetched hold finite values; the padding
+    // columns are never read
     for (int i = threadIdx.x; i < (int)(sizeof(sm.stage) / 16); i += kThreads)
         reinterpret_cast<uint4*>(sm.stage)[i] = make_uint4(0, 0, 0, 0);
     __syncthreads();
@@ -194,92 +215,74 @@ sparse_mla_mma_kernel(const Params p) {
         // ================================ gather ================================
         const int gw = warp - kGatherWarp0;
         const bool leader = gw == 0 && lane == 0;
-        int issued = 0;  // units whose query and indices have been requested
-        auto issue_unit = [&](bool blocking) {
-            const int u2 = blockIdx.x + issued * gridDim.x;
-            if (u2 >= p.num_units) return;
-            const int b2 = issued & 1;
-            const uint32_t par = ((issued >> 1) & 1) ^ 1;
-            if (!blocking && !mbar_try_wait(&sm.q_empty[b2], par)) return;
-            if (blocking) wait_soft(&sm.q_empty[b2], par, abort, p.err);
-            const Unit y = unit_of(p, u2);
-            const uint32_t ibytes = (uint32_t)(y.e1 - y.e0) * 4u;
-            mbar_arrive_expect_tx(&sm.q_full[b2], kH * kDqk * 2 + ibytes);
-            for (int h = 0; h < kH; ++h)
-                bulk_load(sm.q[b2] + h * kQPitch, p.q + ((long long)y.n * kH + h) * kDqk, kDqk * 2,
-                          &sm.q_full[b2]);
-            if (ibytes)
-                bulk_load(sm.idx[b2], p.idx + (long long)y.n * p.ld_idx + y.e0, ibytes,
-                          &sm.q_full[b2]);
-            ++issued;
-        };
         uint32_t G = 0;
-        for (int ui = 0;; ++ui) {
+        int units = 0;
+        for (int ui = 0;; ++ui, ++units) {
             const int u = blockIdx.x + ui * gridDim.x;
             if (u >= p.num_units) break;
             const Unit x = unit_of(p, u);
-            const int qb = ui & 1;
             if (leader) {
-                while (issued <= ui) issue_unit(true);
-                issue_unit(false);
+                // the query of this unit, once the compute warps hold the previous one in
+                // registers
+                wait_soft(&sm.q_empty, (ui & 1) ^ 1, abort, p.err);
+                mbar_arrive_expect_tx(&sm.q_full, kH * kDqk * 2);
+                for (int h = 0; h < kH; ++h)
+                    bulk_load(sm.q + h * kQPitch, p.q + ((long long)x.n * kH + h) * kDqk, kDqk * 2,
+                              &sm.q_full);
             }
-            wait_soft(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err);
-            const int* uidx = sm.idx[qb];
+            // this lane's selected key for the first block; later ones are prefetched a
+            // block ahead
+            int s_next = lane < 16 ? load_index(p, x, x.e0 + gw * 16 + lane) : -1;
             for (int j = 0; j < x.nb; ++j, ++G) {
                 const int s = G & 1;
+                const int s_cur = s_next;
+                if (lane < 16 && j + 1 < x.nb)
+                    s_next = load_index(p, x, x.e0 + (j + 1) * kBK + gw * 16 + lane);
+                const long long row = lane < 16 ? resolve_row(p, x, s_cur) : -1;
                 wait_soft(&sm.a_free[s], ((G >> 1) & 1) ^ 1, abort, p.err);
-                long long row = -1;
-                if (lane < 16) row = resolve_row(p, x, uidx, x.e0 + j * kBK + gw * 16 + lane, true);
-                const uint32_t base = smem_u32(sm.stage[s]) + lane * 16;
-                const char* kvb = reinterpret_cast<const char*>(p.kv) + lane * 16;
-#pragma unroll 4
-                for (int kl = 0; kl < 16; ++kl) {
-                    const long long rr = __shfl_sync(0xffffffffu, row, kl);
-                    const uint32_t dst = base + (gw * 16 + kl) * kRowPitch;
-                    if (rr >= 0) {
-                        const char* src = kvb + rr * (kDqk * 2);
-                        cp_async_16(dst, src);
-                        cp_async_16(dst + 512, src + 512);
-                        if (lane < 8) cp_async_16(dst + 1024, src + 1024);
-                    } else {
-                        cp_async_16_zero(dst, p.kv);
-                        cp_async_16_zero(dst + 512, p.kv);
-                        if (lane < 8) cp_async_16_zero(dst + 1024, p.kv);
-                    }
-                }
-                cp_async_mbar_arrive(&sm.a_full[s]);
-                if (leader && issued == ui + 1) issue_unit(false);
+                if (lane < 16) sm.valid[s][gw * 16 + lane] = row >= 0 ? 1 : -1;
+                const unsigned vmask = __ballot_sync(0xffffffffu, row >= 0);
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive_expect_tx(&sm.a_full[s], (uint32_t)__popc(vmask) * (kDqk * 2));
+                __syncwarp();
+                if (row >= 0)
+                    bulk_load(sm.stage[s] + (gw * 16 + lane) * kRowPitch, p.kv + row * kDqk,
+                              kDqk * 2, &sm.a_full[s]);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.q_empty[qb]);
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
+        // The compute warps consume every block and query, but after a timed-out wait they
+        // may not have: let the last copies land (time-bounded, whatever the abort flag
+        // says) before the CTA can exit.
+        volatile int keep_waiting = 0;
+        for (uint32_t Gl = G >= 2 ? G - 2 : 0; Gl < G; ++Gl)
+            (void)mbar_wait(&sm.a_full[Gl & 1], (Gl >> 1) & 1, &keep_waiting, p.err);
+        if (leader && units > 0) (void)mbar_wait(&sm.q_full, (units - 1) & 1, &keep_waiting, p.err);
     } else {
         // ================================ compute ===============================
-        const int kg = warp & 3;   // key group: keys 16*kg .. 16*kg+15 of a block
-        const int kh = warp >> 2;  // K-half of the QK product
-        const int g = lane >> 2;   // fragment row group
-        const int t = lane & 3;    // thread in group
+        // warp w: K-quarter w of the QK product over all kBK keys, then the softmax of keys
+        // 8w..8w+7 (n-tile w) and PV for output dims kDvWarp*w ..
+        const int g = lane >> 2;    // fragment row group
+        const int t = lane & 3;     // thread in group
         uint32_t G = 0;
         for (int ui = 0;; ++ui) {
             const int u = blockIdx.x + ui * gridDim.x;
             if (u >= p.num_units) break;
             const Unit x = unit_of(p, u);
-            const int qb = ui & 1;
-            wait_soft(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err);
-            const int* uidx = sm.idx[qb];
-            // this warp's K-half of Q as A fragments (16 heads x 16 dims per K-step)
-            uint32_t qa[kKHalf][4];
+            wait_soft(&sm.q_full, ui & 1, abort, p.err);
+            uint32_t qa[kKQuarter][4];
             {
                 const int head = (lane & 7) + ((lane >> 3) & 1) * 8;
-                const uint32_t qrow = smem_u32(sm.q[qb]) + head * kQPitch + ((lane >> 4) & 1) * 16;
+                const uint32_t qrow = smem_u32(sm.q) + head * kQPitch + ((lane >> 4) & 1) * 16;
 #pragma unroll
-                for (int ks = 0; ks < kKHalf; ++ks)
-                    ldsm_x4(qrow + (kh * kKHalf + ks) * 32, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+                for (int ks = 0; ks < kKQuarter; ++ks)
+                    ldsm_x4(qrow + (warp * kKQuarter + ks) * 32, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
             }
-            float o[8][4];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.q_empty);
+            float o[kPVTiles][4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+            for (int i = 0; i < kPVTiles; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
             float m_run[2] = {-INFINITY, -INFINITY};  // heads g, g+8 (log2 domain)
             float l_run[2] = {0.f, 0.f};              // this thread's partial row sums
             float l_lse[2] = {0.f, 0.f};              // the same before bf16 rounding
@@ -288,109 +291,102 @@ sparse_mla_mma_kernel(const Params p) {
                 const int s = G & 1;
                 wait_soft(&sm.a_full[s], (G >> 1) & 1, abort, p.err);
                 const uint32_t st = smem_u32(sm.stage[s]);
-                // ---- QK: S[16 heads x 16 keys] over this warp's K-half ----
-                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                {
-                    const int key = kg * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-                    const uint32_t krow = st + key * kRowPitch + ((lane >> 3) & 1) * 16;
+                // ---- QK: S[16 heads x kBK keys] over this warp's K-quarter ----
+                float acc[kNT][4];
 #pragma unroll
-                    for (int ks = 0; ks < kKHalf; ++ks) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4(krow + (kh * kKHalf + ks) * 32, b0, b1, b2, b3);
-                        mma_bf16(acc[0], qa[ks], b0, b1);
-                        mma_bf16(acc[1], qa[ks], b2, b3);
+                for (int i = 0; i < kNT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+                {
+                    const int key = (lane & 7) + ((lane >> 4) & 1) * 8;
+                    const uint32_t krow = st + key * kRowPitch + ((lane >> 3) & 1) * 16 + warp * kKQuarter * 32;
+#pragma unroll
+                    for (int ks = 0; ks < kKQuarter; ++ks) {
+#pragma unroll
+                        for (int n2 = 0; n2 < kNT / 2; ++n2) {
+                            uint32_t b0, b1, b2, b3;
+                            ldsm_x4(krow + n2 * 16 * kRowPitch + ks * 32, b0, b1, b2, b3);
+                            mma_bf16(acc[2 * n2], qa[ks], b0, b1);
+                            mma_bf16(acc[2 * n2 + 1], qa[ks], b2, b3);
+                        }
                     }
                 }
-                if (kh == 1) {
-                    float4* dst = reinterpret_cast<float4*>(sm.spart[kg][lane]);
-                    dst[0] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-                    dst[1] = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
+                // partial sums of the other warps' n-tiles go through shared memory
+#pragma unroll
+                for (int nt = 0; nt < kNT; ++nt)
+                    if (nt != warp)
+                        *reinterpret_cast<float4*>(sm.spart[warp][nt][lane]) =
+                            make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+                compute_sync();
+                float sc[4];
+                {
+                    float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int nt = 0; nt < kNT; ++nt)
+                        if (nt == warp) { a4[0] = acc[nt][0]; a4[1] = acc[nt][1]; a4[2] = acc[nt][2]; a4[3] = acc[nt][3]; }
+#pragma unroll
+                    for (int w2 = 0; w2 < kComputeWarps; ++w2) {
+                        if (w2 == warp) continue;
+                        const float4 v = *reinterpret_cast<const float4*>(sm.spart[w2][warp][lane]);
+                        a4[0] += v.x; a4[1] += v.y; a4[2] += v.z; a4[3] += v.w;
+                    }
+                    // fragment i: head g + 8*(i>>1), key 8*warp + 2t + (i&1)
+                    const int2 vr = *reinterpret_cast<const int2*>(&sm.valid[s][warp * 8 + 2 * t]);
+                    sc[0] = vr.x >= 0 ? a4[0] * p.scale_log2 : -INFINITY;
+                    sc[1] = vr.y >= 0 ? a4[1] * p.scale_log2 : -INFINITY;
+                    sc[2] = vr.x >= 0 ? a4[2] * p.scale_log2 : -INFINITY;
+                    sc[3] = vr.y >= 0 ? a4[3] * p.scale_log2 : -INFINITY;
+                }
+                float mx0 = fmaxf(sc[0], sc[1]), mx1 = fmaxf(sc[2], sc[3]);
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                if (t == 0) {
+                    sm.red[s][warp][g] = mx0;
+                    sm.red[s][warp][g + 8] = mx1;
                 }
                 compute_sync();
-                if (kh == 0) {
-                    const float4* src = reinterpret_cast<const float4*>(sm.spart[kg][lane]);
-                    const float4 x0 = src[0], x1 = src[1];
-                    acc[0][0] += x0.x; acc[0][1] += x0.y; acc[0][2] += x0.z; acc[0][3] += x0.w;
-                    acc[1][0] += x1.x; acc[1][1] += x1.y; acc[1][2] += x1.z; acc[1][3] += x1.w;
-                    // fragment (nt, i): head g + 8*(i>>1), key 16*kg + 8*nt + 2t + (i&1)
-                    float sv[2][4];
+                float ref[2], alpha[2];
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
+                for (int r = 0; r < 2; ++r) {
+                    float bm = sm.red[s][0][g + 8 * r];
 #pragma unroll
-                        for (int c = 0; c < 2; ++c) {
-                            const int e = x.e0 + j * kBK + kg * 16 + nt * 8 + 2 * t + c;
-                            const bool valid = resolve_row(p, x, uidx, e, false) >= 0;
-                            sv[nt][c] = valid ? acc[nt][c] * p.scale_log2 : -INFINITY;
-                            sv[nt][2 + c] = valid ? acc[nt][2 + c] * p.scale_log2 : -INFINITY;
-                        }
-                    }
-                    // per-head maximum over this warp's 16 keys (rows g and g+8)
-                    float mx0 = fmaxf(fmaxf(sv[0][0], sv[0][1]), fmaxf(sv[1][0], sv[1][1]));
-                    float mx1 = fmaxf(fmaxf(sv[0][2], sv[0][3]), fmaxf(sv[1][2], sv[1][3]));
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-                    if (t == 0) {
-                        sm.red[kg][g] = mx0;
-                        sm.red[kg][g + 8] = mx1;
-                    }
-                    named_bar_sync(2, 128);  // the four K-half-0 warps
-                    float bm[2];
-                    bm[0] = fmaxf(fmaxf(sm.red[0][g], sm.red[1][g]), fmaxf(sm.red[2][g], sm.red[3][g]));
-                    bm[1] = fmaxf(fmaxf(sm.red[0][g + 8], sm.red[1][g + 8]),
-                                  fmaxf(sm.red[2][g + 8], sm.red[3][g + 8]));
-                    float alpha[2], ref[2];
-#pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const float mn = fmaxf(m_run[r], bm[r]);
-                        alpha[r] = m_run[r] == -INFINITY ? 0.f : exp2f(m_run[r] - mn);
-                        m_run[r] = mn;
-                        ref[r] = mn == -INFINITY ? 0.f : mn;  // no valid key yet: P = 0 anyway
-                        l_run[r] *= alpha[r];
-                        l_lse[r] *= alpha[r];
-                    }
-                    // P = exp2(s - m) in bf16; invalid keys (s = -inf) give exactly 0
-                    uint8_t* pb = sm.p[s];
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-                        for (int r = 0; r < 2; ++r) {
-                            const float p0 = exp2f(sv[nt][2 * r] - ref[r]);
-                            const float p1 = exp2f(sv[nt][2 * r + 1] - ref[r]);
-                            const uint32_t pk = pack_bf16(p0, p1);
-                            const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&pk);
-                            l_run[r] += __bfloat162float(pr.x) + __bfloat162float(pr.y);
-                            l_lse[r] += p0 + p1;
-                            const int head = g + 8 * r;
-                            const int key = kg * 16 + nt * 8 + 2 * t;
-                            *reinterpret_cast<uint32_t*>(pb + head * kPPitch + key * 2) = pk;
-                        }
-                    }
-                    if (kg == 0 && t == 0) {
-                        sm.alpha[g] = alpha[0];
-                        sm.alpha[g + 8] = alpha[1];
-                    }
+                    for (int i = 1; i < kComputeWarps; ++i) bm = fmaxf(bm, sm.red[s][i][g + 8 * r]);
+                    const float mn = fmaxf(m_run[r], bm);
+                    alpha[r] = m_run[r] == -INFINITY ? 0.f : exp2f(m_run[r] - mn);
+                    m_run[r] = mn;
+                    ref[r] = mn == -INFINITY ? 0.f : mn;  // no valid key yet: P = 0 anyway
+                    l_run[r] *= alpha[r];
+                    l_lse[r] *= alpha[r];
                 }
-                compute_sync();  // P and alpha of this block are in shared memory
-                // ---- PV: O[16 heads x 64 dims of this warp] += P[16 x 64 keys] V ----
-                {
-                    const float a0 = sm.alpha[g], a1 = sm.alpha[g + 8];
+                // P = exp2(s - m) in bf16; invalid keys (s = -inf) give exactly 0
 #pragma unroll
-                    for (int n = 0; n < 8; ++n) {
-                        o[n][0] *= a0; o[n][1] *= a0;
-                        o[n][2] *= a1; o[n][3] *= a1;
-                    }
+                for (int r = 0; r < 2; ++r) {
+                    const float p0 = exp2f(sc[2 * r] - ref[r]);
+                    const float p1 = exp2f(sc[2 * r + 1] - ref[r]);
+                    const uint32_t pk = pack_bf16(p0, p1);
+                    const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&pk);
+                    l_run[r] += __bfloat162float(pr.x) + __bfloat162float(pr.y);
+                    l_lse[r] += p0 + p1;
+                    *reinterpret_cast<uint32_t*>(sm.p[s] + (g + 8 * r) * kPPitch + (warp * 8 + 2 * t) * 2) = pk;
+                }
+#pragma unroll
+                for (int n = 0; n < kPVTiles; ++n) {
+                    o[n][0] *= alpha[0]; o[n][1] *= alpha[0];
+                    o[n][2] *= alpha[1]; o[n][3] *= alpha[1];
+                }
+                compute_sync();  // P of this block is in shared memory
+                // ---- PV: O[16 heads x kDvWarp dims of this warp] += P[16 x kBK keys] V ----
+                {
                     const int head = (lane & 7) + ((lane >> 3) & 1) * 8;
                     const uint32_t prow = smem_u32(sm.p[s]) + head * kPPitch + ((lane >> 4) & 1) * 16;
                     const int vkey = (lane & 7) + ((lane >> 3) & 1) * 8;
-                    const uint32_t vrow = st + vkey * kRowPitch + (warp * 64 + ((lane >> 4) & 1) * 8) * 2;
+                    const uint32_t vrow = st + vkey * kRowPitch + (warp * kDvWarp + ((lane >> 4) & 1) * 8) * 2;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         uint32_t pa[4];
                         ldsm_x4(prow + kk * 32, pa[0], pa[1], pa[2], pa[3]);
 #pragma unroll
-                        for (int n2 = 0; n2 < 4; ++n2) {
+                        for (int n2 = 0; n2 < kPVTiles / 2; ++n2) {
                             uint32_t b0, b1, b2, b3;
                             ldsm_x4_t(vrow + kk * 16 * kRowPitch + n2 * 32, b0, b1, b2, b3);
                             mma_bf16(o[2 * n2], pa, b0, b1);
@@ -403,44 +399,33 @@ sparse_mla_mma_kernel(const Params p) {
             }
 
             // ---- epilogue of the unit: row sums, normalise, write ----
-            if (kh == 0) {
 #pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
-                    l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
-                    l_lse[r] += __shfl_xor_sync(0xffffffffu, l_lse[r], 1);
-                    l_lse[r] += __shfl_xor_sync(0xffffffffu, l_lse[r], 2);
-                }
-                if (t == 0) {
-                    sm.lsum[kg][g] = l_run[0];
-                    sm.lsum[kg][g + 8] = l_run[1];
-                }
+            for (int r = 0; r < 2; ++r) {
+                l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+                l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+                l_lse[r] += __shfl_xor_sync(0xffffffffu, l_lse[r], 1);
+                l_lse[r] += __shfl_xor_sync(0xffffffffu, l_lse[r], 2);
+            }
+            if (t == 0) {
+                sm.lsum[0][warp][g] = l_run[0];
+                sm.lsum[0][warp][g + 8] = l_run[1];
+                sm.lsum[1][warp][g] = l_lse[0];
+                sm.lsum[1][warp][g + 8] = l_lse[1];
             }
             compute_sync();
-            float L[2], Lx[2] = {0.f, 0.f};
-            L[0] = sm.lsum[0][g] + sm.lsum[1][g] + sm.lsum[2][g] + sm.lsum[3][g];
-            L[1] = sm.lsum[0][g + 8] + sm.lsum[1][g + 8] + sm.lsum[2][g + 8] + sm.lsum[3][g + 8];
-            compute_sync();  // lsum is reused for the exact sums below
-            if (kh == 0 && t == 0) {
-                sm.lsum[kg][g] = l_lse[0];
-                sm.lsum[kg][g + 8] = l_lse[1];
+            float L[2] = {0.f, 0.f}, Lx[2] = {0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < kComputeWarps; ++i) {
+                L[0] += sm.lsum[0][i][g];
+                L[1] += sm.lsum[0][i][g + 8];
+                Lx[0] += sm.lsum[1][i][g];
+                Lx[1] += sm.lsum[1][i][g + 8];
             }
-            compute_sync();
-            Lx[0] = sm.lsum[0][g] + sm.lsum[1][g] + sm.lsum[2][g] + sm.lsum[3][g];
-            Lx[1] = sm.lsum[0][g + 8] + sm.lsum[1][g + 8] + sm.lsum[2][g + 8] + sm.lsum[3][g + 8];
-            // m_run is only kept by the K-half-0 warps; broadcast it through alpha's slot
-            compute_sync();
-            if (kh == 0 && kg == 0 && t == 0) {
-                sm.alpha[g] = m_run[0];
-                sm.alpha[g + 8] = m_run[1];
-            }
-            compute_sync();
-            const float mr[2] = {sm.alpha[g], sm.alpha[g + 8]};
             const float inv0 = (x.nb > 0 && L[0] > 0.f) ? 1.f / L[0] : 0.f;
             const float inv1 = (x.nb > 0 && L[1] > 0.f) ? 1.f / L[1] : 0.f;
 #pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const int dim = warp * 64 + n * 8 + 2 * t;
+            for (int n = 0; n < kPVTiles; ++n) {
+                const int dim = warp * kDvWarp + n * 8 + 2 * t;
                 if (p.page_table == nullptr) {
                     __nv_bfloat16* o0 = p.out + ((long long)x.n * kH + g) * kDv + dim;
                     __nv_bfloat16* o1 = p.out + ((long long)x.n * kH + g + 8) * kDv + dim;
@@ -457,7 +442,7 @@ sparse_mla_mma_kernel(const Params p) {
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
                     const int head = g + 8 * r;
-                    const float l = (x.nb > 0 && Lx[r] > 0.f) ? (mr[r] + log2f(Lx[r])) * 0.69314718055994531f
+                    const float l = (x.nb > 0 && Lx[r] > 0.f) ? (m_run[r] + log2f(Lx[r])) * 0.69314718055994531f
                                                            : -INFINITY;
                     if (p.page_table == nullptr) {
                         if (p.lse != nullptr) p.lse[(long long)x.n * kH + head] = l;
@@ -466,8 +451,7 @@ sparse_mla_mma_kernel(const Params p) {
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.q_empty[qb]);
+            compute_sync();  // lsum is rewritten by the next unit
         }
     }
 }
@@ -549,7 +533,12 @@ cudaError_t launch_sparse_mla_mma(const __nv_bfloat16* q, const __nv_bfloat16* k
     cudaError_t e = cudaFuncSetAttribute(sparse_mla_mma_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int grid = p.num_units < ctx.num_sms ? p.num_units : ctx.num_sms;
+    // two CTAs per SM need most of the shared memory carve-out
+    e = cudaFuncSetAttribute(sparse_mla_mma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    const int slots = kCtasPerSm * ctx.num_sms;
+    const int grid = p.num_units < slots ? p.num_units : slots;
     sparse_mla_mma_kernel<<<grid, kThreads, smem, stream>>>(p);
     count_launch(DSA_KERNEL_ATTENTION);
     return cudaGetLastError();
