@@ -230,15 +230,19 @@ sparse_mla_mma_kernel(const Params p) {
                     bulk_load(sm.q + h * kQPitch, p.q + ((long long)x.n * kH + h) * kDqk, kDqk * 2,
                               &sm.q_full);
             }
-            // this lane's selected key for the first block; later ones are prefetched a
-            // block ahead
-            int s_next = lane < 16 ? load_index(p, x, x.e0 + gw * 16 + lane) : -1;
+            // This lane's selected keys are read two blocks ahead of their copies and
+            // resolved to cache rows (a page-table load in decode) one block ahead.
+            const int e_lane = x.e0 + gw * 16 + lane;
+            int s_ahead = lane < 16 ? load_index(p, x, e_lane + kBK) : -1;
+            long long row_next = lane < 16 ? resolve_row(p, x, load_index(p, x, e_lane)) : -1;
             for (int j = 0; j < x.nb; ++j, ++G) {
                 const int s = G & 1;
-                const int s_cur = s_next;
-                if (lane < 16 && j + 1 < x.nb)
-                    s_next = load_index(p, x, x.e0 + (j + 1) * kBK + gw * 16 + lane);
-                const long long row = lane < 16 ? resolve_row(p, x, s_cur) : -1;
+                const long long row = row_next;
+                if (lane < 16) {
+                    const int s_far = load_index(p, x, e_lane + (j + 2) * kBK);
+                    row_next = resolve_row(p, x, s_ahead);
+                    s_ahead = s_far;
+                }
                 wait_soft(&sm.a_free[s], ((G >> 1) & 1) ^ 1, abort, p.err);
                 if (lane < 16) sm.valid[s][gw * 16 + lane] = row >= 0 ? 1 : -1;
                 const unsigned vmask = __ballot_sync(0xffffffffu, row >= 0);
@@ -491,13 +495,28 @@ __global__ void mla_combine_kernel(const float* __restrict__ o_part,
 
 }  // namespace
 
+// Splits per decode sequence: the count that minimises the modelled time, waves of units
+// over the CTA slots times (key blocks per unit + a per-unit start-up cost of about four
+// blocks: the query copy and the first gather round trip); ties go to fewer splits.
 int mla_decode_splits(int num_q, int k_sel, int num_sms) {
+    constexpr int kUnitStartBlocks = 4;
     const int blocks = (k_sel + kBK - 1) / kBK;
-    int splits = (4 * num_sms + num_q - 1) / (num_q > 0 ? num_q : 1);
-    if (splits < 1) splits = 1;
-    if (splits > blocks) splits = blocks;
-    const int chunk = ((k_sel + splits - 1) / splits + kBK - 1) / kBK * kBK;
-    return (k_sel + chunk - 1) / chunk;
+    const long long slots = (long long)kCtasPerSm * num_sms;
+    const int nq = num_q > 0 ? num_q : 1;
+    int best = 1;
+    long long best_cost = -1;
+    for (int sp = 1; sp <= blocks; ++sp) {
+        const int per_unit = (blocks + sp - 1) / sp;
+        const int splits = (blocks + per_unit - 1) / per_unit;  // no empty split
+        if (splits != sp) continue;
+        const long long waves = ((long long)nq * splits + slots - 1) / slots;
+        const long long cost = waves * (per_unit + kUnitStartBlocks);
+        if (best_cost < 0 || cost < best_cost) {
+            best = splits;
+            best_cost = cost;
+        }
+    }
+    return best;
 }
 
 size_t mla_mma_smem_bytes() { return sizeof(MmaSmem) + 128; }

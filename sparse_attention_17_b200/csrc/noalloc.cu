@@ -77,11 +77,11 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(
     if (e != cudaSuccess) return DSA_ERR_CUDA;
     void* scratch = nullptr;
     if (scratch_address(&scratch) != cudaSuccess) return DSA_ERR_CUDA;
-    // as many splits as the usual path would take, capped by what the array holds
+    // as many splits as the usual path would take, capped by what the array holds (a
+    // trailing split left without keys writes a zero partial with log-sum-exp -inf, which
+    // the merge ignores)
     int splits = mla_decode_splits(num_q, k_sel, ctx.num_sms);
     if (splits > kMaxUnits / num_q) splits = kMaxUnits / num_q;
-    const int chunk = ((k_sel + splits - 1) / splits + 63) / 64 * 64;
-    splits = (k_sel + chunk - 1) / chunk;
     float* o_part = static_cast<float*>(scratch);
     float* lse_part = o_part + (size_t)num_q * splits * 16 * 512;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);

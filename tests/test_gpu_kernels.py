@@ -263,8 +263,8 @@ def test_topk_sample_miss_falls_back_to_exact():
 
 def test_topk_one_warp_region_overflows_to_exact():
     """Every large score sits in 128-key chunks that one warp of the candidate pass reads
-    (chunk index = 3 mod 16), and the threshold sample never reads those chunks: that
-    warp's candidate slice overflows and the row must be redone exactly."""
+    (chunk index = 3 mod 16, so 3 mod 8 as well): that warp's candidate slice overflows
+    and the row must be redone exactly."""
     S, k = 65536, 2048
     r = np.random.default_rng(11)
     sc = r.normal(size=(2, S))
@@ -275,9 +275,11 @@ def test_topk_one_warp_region_overflows_to_exact():
     check_indices_exact(idx, ref, "one-warp overflow")
 
 
-@pytest.mark.parametrize("n_valid", [[8192, 8193, 8191, 12345, 2049, 65536, 16385, 4097]])
+@pytest.mark.parametrize("n_valid", [[3072, 3073, 3071, 8192, 8193, 12345, 2049, 65536, 16385,
+                                      4097, 3840, 3841]])
 def test_topk_lengths_around_sample_switch(n_valid):
-    """Rows of at most 8192 keys skip the threshold sample; longer ones use it."""
+    """Rows of at most 3072 keys skip the threshold sample (every key is a candidate);
+    longer ones use it."""
     S, k = 65536, 2048
     r = np.random.default_rng(12)
     sc = r.normal(size=(len(n_valid), S)).astype(np.float32).astype(np.float64)
