@@ -5,19 +5,18 @@
 // n <= k every key is selected.  Output: the selected key positions in ascending order,
 // then -1 padding.
 //
-// One CTA of 256 threads per row, four CTAs per SM (rows in flight hide the latency of the
-// block-wide radix rounds).  Scores map to order-preserving uint32 keys.  Each warp owns a
-// 480-entry slice of the shared candidate buffer, so candidates are appended with
+// One CTA of 512 threads per row.  Scores map to order-preserving uint32 keys.  Each warp
+// owns a 512-entry slice of the shared candidate buffer, so candidates are appended with
 // a ballot and a popcount and no shared atomics.
 // Fast path (one read of the row):
-//   sample  a strided sample of 32-key chunks of the row (at most 120 chunks, every 16th
-//           or sparser, all loads in flight at once) goes to the slices; a two-round
-//           (11 + 11 bit) radix select there gives a provisional threshold tau0 below the
-//           sample rank that corresponds to k plus a few standard deviations (rows of at
-//           most 3072 keys skip this: tau0 = the smallest key);
+//   sample  every 16th 32-key chunk of the row (at most 256 chunks, all loads in flight
+//           at once) goes to the slices; a two-round (12 + 12 bit) radix select there
+//           gives a provisional threshold tau0 below the sample rank that corresponds to
+//           k plus a few standard deviations (rows of at most 8192 keys skip this:
+//           tau0 = the smallest key);
 //   gather  one pass with four 16-byte loads per thread in flight appends every key
 //           >= tau0 to the warp's slice (128-key chunks dealt round-robin to the warps);
-//   select  radix select (11 + 11 + 10 bits) among the candidates gives the k-th largest
+//   select  radix select (12 + 12 + 8 bits) among the candidates gives the k-th largest
 //           key tau; candidates above tau are selected, those equal to tau are ties.
 // If the candidates number fewer than k or more than a slice holds, the row is redone
 // exactly from global memory (histogram passes over the whole row).  Finally the first
@@ -30,16 +29,10 @@ namespace dsa {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-// Radix digits of the 32-bit order keys: 11 + 11 + 10 bits.
-constexpr int kShift1 = 21;                // digit 1: bits 31..21
-constexpr int kShift2 = 10;                // digit 2: bits 20..10
-constexpr uint32_t kMask2 = 0x7FFu;
-constexpr uint32_t kMask3 = 0x3FFu;        // digit 3: bits 9..0
-constexpr int kBins = 2048;                // histogram bins (digits 1 and 2)
-constexpr int kBins3 = 1024;               // histogram bins of digit 3
-constexpr int kCandCap = 3840;
+constexpr int kBins = 4096;
+constexpr int kCandCap = 8192;
 constexpr int kStride = kWarps * 32;  // elements covered by all warps per iteration
 constexpr int kSlice = kCandCap / kWarps;  // candidate entries owned by one warp
 constexpr int kUnroll = 4;                 // 16-byte loads in flight per thread
@@ -55,8 +48,8 @@ struct TopkScratch {
     uint32_t found_above;
 };
 
-constexpr int kSampleChunks = kCandCap / 32;  // at most 120 sampled 32-key chunks
-constexpr int kSampleChunksPerWarp = kSampleChunks / kWarps;  // 15 chunks = one slice
+constexpr int kSampleChunks = kCandCap / 32;  // at most 256 sampled 32-key chunks
+constexpr int kSampleChunksPerWarp = kSampleChunks / kWarps;  // 16 chunks = one slice
 // rows this short make every key a candidate: each warp's 128-key chunks fit its slice
 constexpr int kNoSampleMax = (kSlice / 128) * 128 * kWarps;
 
@@ -133,8 +126,8 @@ __device__ __forceinline__ void zero_hist(TopkScratch& sh, int nbins) {
 
 // Radix select over the warps' candidate slices (warp w owns cand_key[w * kSlice ..] with
 // wcount[w] <= kSlice entries).  exact: returns the need-th largest key tau and sets
-// *need_out to how many keys equal to tau belong to the top `need` (all three digits).
-// !exact: stops after two digits and returns the lower edge of the 22-bit bin holding the
+// *need_out to how many keys equal to tau belong to the top `need` (12 + 12 + 8 bits).
+// !exact: stops after 24 bits and returns the lower edge of the 24-bit bin holding the
 // need-th largest key, a lower bound of it.
 __device__ uint32_t slice_radix_select(TopkScratch& sh, uint32_t need, bool exact,
                                        uint32_t* need_out) {
@@ -145,7 +138,7 @@ __device__ uint32_t slice_radix_select(TopkScratch& sh, uint32_t need, bool exac
     __syncthreads();
     for (int c0 = 0; c0 < cnt; c0 += 32) {
         const int c = c0 + lane;
-        hist_add(sh.hist, c < cnt ? keys[c] >> kShift1 : 0u, c < cnt);
+        hist_add(sh.hist, c < cnt ? keys[c] >> 20 : 0u, c < cnt);
     }
     __syncthreads();
     find_bin(sh, kBins, need);
@@ -156,29 +149,29 @@ __device__ uint32_t slice_radix_select(TopkScratch& sh, uint32_t need, bool exac
     for (int c0 = 0; c0 < cnt; c0 += 32) {
         const int c = c0 + lane;
         const uint32_t key = c < cnt ? keys[c] : 0u;
-        hist_add(sh.hist, (key >> kShift2) & kMask2, c < cnt && (key >> kShift1) == b1);
+        hist_add(sh.hist, (key >> 8) & 0xFFFu, c < cnt && (key >> 20) == b1);
     }
     __syncthreads();
     find_bin(sh, kBins, need);
-    const uint32_t pre = (b1 << (kShift1 - kShift2)) | sh.found_bin;
+    const uint32_t pre = (b1 << 12) | sh.found_bin;
     need -= sh.found_above;
     if (!exact) {
         *need_out = need;
         __syncthreads();
-        return pre << kShift2;
+        return pre << 8;
     }
-    zero_hist(sh, kBins3);
+    zero_hist(sh, 256);
     __syncthreads();
     for (int c0 = 0; c0 < cnt; c0 += 32) {
         const int c = c0 + lane;
         const uint32_t key = c < cnt ? keys[c] : 0u;
-        hist_add(sh.hist, key & kMask3, c < cnt && (key >> kShift2) == pre);
+        hist_add(sh.hist, key & 0xFFu, c < cnt && (key >> 8) == pre);
     }
     __syncthreads();
-    find_bin(sh, kBins3, need);
+    find_bin(sh, 256, need);
     need -= sh.found_above;
     *need_out = need;
-    const uint32_t tau = (pre << kShift2) | sh.found_bin;
+    const uint32_t tau = (pre << 8) | sh.found_bin;
     __syncthreads();
     return tau;
 }
@@ -203,7 +196,7 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
             x[u] = in[u] ? __ldg(row + s) : 0.f;
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) hist_add(sh.hist, float_order_key(x[u]) >> kShift1, in[u]);
+        for (int u = 0; u < 4; ++u) hist_add(sh.hist, float_order_key(x[u]) >> 20, in[u]);
     }
     __syncthreads();
     find_bin(sh, kBins, (uint32_t)k);
@@ -219,7 +212,7 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
             const int s = base + lane;
             const bool in = s < n;
             const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
-            const uint32_t hi = key >> kShift1;
+            const uint32_t hi = key >> 20;
             const unsigned gt = __ballot_sync(0xffffffffu, in && hi > b1);
             const bool eq = in && hi == b1;
             const unsigned meq = __ballot_sync(0xffffffffu, eq);
@@ -242,26 +235,26 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
         for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
             const int c = c0 + lane;
             const bool in = c < cnt;
-            hist_add(sh.hist, in ? (sh.cand_key[c] >> kShift2) & kMask2 : 0u, in);
+            hist_add(sh.hist, in ? (sh.cand_key[c] >> 8) & 0xFFFu : 0u, in);
         }
         __syncthreads();
         find_bin(sh, kBins, need);
         const uint32_t b2 = sh.found_bin;
         need -= sh.found_above;
-        zero_hist(sh, kBins3);
+        zero_hist(sh, 256);
         __syncthreads();
         // ---- refine: bits 7..0 ----
-        const uint32_t pre = (b1 << (kShift1 - kShift2)) | b2;
+        const uint32_t pre = (b1 << 12) | b2;
         for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
             const int c = c0 + lane;
             const uint32_t key = c < cnt ? sh.cand_key[c] : 0u;
-            const bool in = c < cnt && (key >> kShift2) == pre;
-            hist_add(sh.hist, key & kMask3, in);
+            const bool in = c < cnt && (key >> 8) == pre;
+            hist_add(sh.hist, key & 0xFFu, in);
         }
         __syncthreads();
-        find_bin(sh, kBins3, need);
+        find_bin(sh, 256, need);
         need -= sh.found_above;
-        tau = (pre << kShift2) | sh.found_bin;
+        tau = (pre << 8) | sh.found_bin;
         for (int c = threadIdx.x; c < cnt; c += kThreads) {
             const uint32_t key = sh.cand_key[c];
             const int s = sh.cand_idx[c];
@@ -276,25 +269,25 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
             const int s = base + lane;
             const bool in = s < n;
             const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
-            hist_add(sh.hist, (key >> kShift2) & kMask2, in && (key >> kShift1) == b1);
+            hist_add(sh.hist, (key >> 8) & 0xFFFu, in && (key >> 20) == b1);
         }
         __syncthreads();
         find_bin(sh, kBins, need);
         const uint32_t b2 = sh.found_bin;
         need -= sh.found_above;
-        zero_hist(sh, kBins3);
+        zero_hist(sh, 256);
         __syncthreads();
-        const uint32_t pre = (b1 << (kShift1 - kShift2)) | b2;
+        const uint32_t pre = (b1 << 12) | b2;
         for (int base = warp * 32; base < n; base += kStride) {
             const int s = base + lane;
             const bool in = s < n;
             const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
-            hist_add(sh.hist, key & kMask3, in && (key >> kShift2) == pre);
+            hist_add(sh.hist, key & 0xFFu, in && (key >> 8) == pre);
         }
         __syncthreads();
-        find_bin(sh, kBins3, need);
+        find_bin(sh, 256, need);
         need -= sh.found_above;
-        tau = (pre << kShift2) | sh.found_bin;
+        tau = (pre << 8) | sh.found_bin;
         for (int base = warp * 32; base < n; base += kStride) {
             const int s = base + lane;
             const bool in = s < n;
@@ -311,7 +304,7 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
     return need;
 }
 
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kThreads, 2)
 topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
                   const int* __restrict__ row_len, int max_len, int k, int* __restrict__ idx,
                   long long ld_idx, unsigned* __restrict__ err) {

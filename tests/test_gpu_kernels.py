@@ -278,7 +278,7 @@ def test_topk_one_warp_region_overflows_to_exact():
 @pytest.mark.parametrize("n_valid", [[3072, 3073, 3071, 8192, 8193, 12345, 2049, 65536, 16385,
                                       4097, 3840, 3841]])
 def test_topk_lengths_around_sample_switch(n_valid):
-    """Rows of at most 3072 keys skip the threshold sample (every key is a candidate);
+    """Rows of at most 8192 keys skip the threshold sample (every key is a candidate);
     longer ones use it."""
     S, k = 65536, 2048
     r = np.random.default_rng(12)
