@@ -136,6 +136,38 @@ dsa_status dsa_topk_select(const float* scores, long long ld_scores, int rows, i
                            long long ld_idx, dsa_stream_t stream);
 
 /*
+ * dsa_index_select -- lightning-indexer scores and the per-row top-k of causal prefill rows
+ * in one call, without writing the dense score rows (DSA ablation card, "Attention" bullet:
+ * every key is scored, the top-k keys are kept).  The result is identical to
+ * dsa_indexer_scores (bf16, prefill) followed by dsa_topk_select on the same rows: the same
+ * tensor-core scores, the same selection rule and ties, the same output layout.
+ *
+ * Method: per window of rows, one 128-key tile in 16 is scored first and each row gets a
+ * threshold a few standard deviations below the score its k-th largest key is expected to
+ * have; the full scoring pass then appends only the keys above the threshold to per-row
+ * candidate lists and marks the keys equal to it in a bitmap; the exact top-k is taken among
+ * those.  A row the candidates cannot settle (too many, or too few together with the
+ * ties) is recomputed from dense scores of its window, so the result never depends on the
+ * sample.
+ *
+ * q_idx [q_begin+rows, 16, 64] bf16 (query t in row t), k_idx [S, 64] bf16, w [q_begin+rows,
+ * 16] fp32; query row t = q_begin + r has the n = t + 1 keys 0..t (q_begin + rows <= S <=
+ * 262144).  idx [rows, ld_idx] int32 receives, per row, the selected key positions in
+ * ascending order then -1 padding (1 <= k <= 4096, ld_idx >= k, a multiple of 4).
+ * workspace: caller-owned device scratch, 256-byte aligned; rows are processed in windows
+ * of the largest multiple of 16 rows (or all rows) for which
+ * dsa_index_select_workspace_size(window, S) <= ws_bytes; fewer than 16 rows ->
+ * DSA_ERR_WORKSPACE.  Supported: H_I = 16, D_I = 64 (else DSA_ERR_UNSUPPORTED).
+ */
+dsa_status dsa_index_select(const void* q_idx, const void* k_idx, const float* w, int H_I,
+                            int D_I, int q_begin, int rows, int S, int k, int* idx,
+                            long long ld_idx, void* workspace, size_t ws_bytes,
+                            dsa_stream_t stream);
+
+/* Scratch bytes dsa_index_select needs for a window of rows_window rows and S keys. */
+size_t dsa_index_select_workspace_size(int rows_window, int S);
+
+/*
  * dsa_sparse_mla_fwd -- attention over the selected keys only (DSV2-Lite-IndexCache card:
  * attention_mode="sparse"; its portable runtime is the same computation as masked SDPA).
  *

@@ -32,6 +32,8 @@ SYMBOLS = [
     ("dsa_version", _I, []),
     ("dsa_indexer_scores", _I, [_I, _I, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _I, _P, _P, _LL, _P]),
     ("dsa_topk_select", _I, [_P, _LL, _I, _I, _P, _I, _I, _P, _LL, _P]),
+    ("dsa_index_select", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _LL, _P, _SZ, _P]),
+    ("dsa_index_select_workspace_size", _SZ, [_I, _I]),
     ("dsa_sparse_mla_fwd", _I, [_I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _LL, _P, _I, _I, _P,
                                 _P, _I, _LL, _P, _P, _P, _SZ, _P]),
     ("dsa_sparse_mla_workspace_size", _SZ, [_I, _I, _I, _I, _I]),
@@ -159,6 +161,30 @@ def topk_select(scores, k: int, idx, q_begin: int = 0, rows: int | None = None, 
     _check(lib.dsa_topk_select(scores.data_ptr(), scores.stride(0), rows, q_begin,
                                _ptr(row_len), max_len, k, idx.data_ptr(), idx.stride(0),
                                _stream()))
+
+
+def index_select_workspace_size(rows_window: int, S: int) -> int:
+    return load().dsa_index_select_workspace_size(rows_window, S)
+
+
+def index_select(q_idx, k_idx, w, idx, k: int, workspace, q_begin: int = 0,
+                 rows: int | None = None) -> None:
+    """dsa_index_select: indexer + top-k of causal prefill rows without dense score rows.
+    q_idx [T,16,64] bf16, k_idx [S,64] bf16, w [T,16] fp32, idx [rows, >=k] int32 (row r is
+    query q_begin + r), workspace a CUDA tensor (any dtype) used as scratch."""
+    lib = load()
+    _need(q_idx, torch.bfloat16, 3, "q_idx")
+    _need(k_idx, torch.bfloat16, 2, "k_idx")
+    _need(w, torch.float32, 2, "w")
+    _need(idx, torch.int32, 2, "idx")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    if rows is None:
+        rows = q_idx.shape[0] - q_begin
+    _check(lib.dsa_index_select(q_idx.data_ptr(), k_idx.data_ptr(), w.data_ptr(), q_idx.shape[1],
+                                q_idx.shape[2], q_begin, rows, k_idx.shape[0], k, idx.data_ptr(),
+                                idx.stride(0), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), _stream()))
 
 
 def sparse_mla_workspace_size(num_q: int, k_sel: int, decode: bool, H: int = 16,

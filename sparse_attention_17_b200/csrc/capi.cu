@@ -323,6 +323,136 @@ size_t dsa_layer_stack_workspace_size(int T, int rows_window) {
     return (size_t)(rw * ld * 4);
 }
 
+// ---- filtered index selection (dsa_index_select) ----
+namespace {
+
+constexpr int kSampleStride = 16;     // one 128-key tile in 16 is scored for the thresholds
+constexpr int kDenseRows = 8192;      // rows with at most this many keys take the dense path
+constexpr int kListCap = 512;         // candidates per (row, 4096-key chunk, lane quadrant)
+
+struct SelectLayout {
+    long long ld_sample, ld_dense, nchunk_max;
+    size_t off_sample, off_tau, off_fb_row, off_fb_any, off_ccount, off_cand, off_dense;
+    size_t total;
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+SelectLayout select_layout(long long rows, long long S) {
+    SelectLayout L{};
+    const long long span = 128LL * kSampleStride;
+    L.ld_sample = (S + span - 1) / span * 128;
+    L.ld_dense = (S + 3) / 4 * 4;
+    L.nchunk_max = (S + 4095) / 4096;
+    const long long lists = rows * L.nchunk_max * 4;
+    size_t o = 0;
+    L.off_sample = o; o = align256(o + (size_t)(rows * L.ld_sample) * 4);
+    L.off_tau = o;    o = align256(o + (size_t)rows * 4);
+    L.off_fb_row = o; o = align256(o + (size_t)rows * 4);
+    L.off_fb_any = o; o = align256(o + 4);
+    L.off_ccount = o; o = align256(o + (size_t)lists * 4);
+    L.off_cand = o;   o = align256(o + (size_t)lists * kListCap * 8);
+    L.off_dense = o;  o = align256(o + (size_t)(rows * L.ld_dense) * 4);
+    L.total = o;
+    return L;
+}
+
+}  // namespace
+
+size_t dsa_index_select_workspace_size(int rows_window, int S) {
+    if (rows_window <= 0 || S <= 0) return 0;
+    return select_layout(rows_window, S).total;
+}
+
+dsa_status dsa_index_select(const void* q_idx, const void* k_idx, const float* w, int H_I, int D_I,
+                            int q_begin, int rows, int S, int k, int* idx, long long ld_idx,
+                            void* workspace, size_t ws_bytes, dsa_stream_t stream) {
+    g_last_error[0] = 0;
+    if (!q_idx || !k_idx || !w || !idx) return fail(DSA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(idx))
+        return fail(DSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (rows < 0 || q_begin < 0 || S <= 0) return fail(DSA_ERR_INVALID_ARG, "bad rows / q_begin / S");
+    if (H_I != 16 || D_I != 64)
+        return fail(DSA_ERR_UNSUPPORTED, "bf16 indexer supports H_I=16, D_I=64 only");
+    if (k < 1 || k > 4096) return fail(DSA_ERR_UNSUPPORTED, "k must be in [1, 4096]");
+    if (ld_idx < k || (ld_idx & 3)) return fail(DSA_ERR_INVALID_ARG, "ld_idx must be >= k and a multiple of 4");
+    if ((long long)q_begin + rows > S)
+        return fail(DSA_ERR_INVALID_ARG, "causal keys 0..q_begin+rows-1 exceed S=%d", S);
+    if ((long long)S > 262144) return fail(DSA_ERR_UNSUPPORTED, "S must be <= 262144");
+    if (rows == 0) return DSA_OK;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return fail(DSA_ERR_INVALID_ARG, "workspace must be non-null and 256-byte aligned");
+    // the largest window (a multiple of 16 rows, or all rows) whose scratch fits
+    long long rw = rows;
+    if (select_layout(rw, S).total > ws_bytes) {
+        long long lo = 0, hi = rows;
+        while (lo < hi) {
+            const long long mid = (lo + hi + 1) / 2;
+            if (select_layout(mid, S).total <= ws_bytes) lo = mid; else hi = mid - 1;
+        }
+        rw = lo / 16 * 16;
+        if (rw < 16) return fail(DSA_ERR_WORKSPACE, "workspace holds fewer than 16 rows");
+    }
+    DevCtx ctx;
+    dsa_status st = check_stream_device(&ctx);
+    if (st != DSA_OK) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const SelectLayout L = select_layout(rw, S);
+    char* base = static_cast<char*>(workspace);
+    float* sample = reinterpret_cast<float*>(base + L.off_sample);
+    uint32_t* tau = reinterpret_cast<uint32_t*>(base + L.off_tau);
+    int* fb_row = reinterpret_cast<int*>(base + L.off_fb_row);
+    int* fb_any = reinterpret_cast<int*>(base + L.off_fb_any);
+    uint32_t* ccount = reinterpret_cast<uint32_t*>(base + L.off_ccount);
+    uint2* cand = reinterpret_cast<uint2*>(base + L.off_cand);
+    float* dense = reinterpret_cast<float*>(base + L.off_dense);
+    const auto* qi = static_cast<const __nv_bfloat16*>(q_idx);
+    const auto* ki = static_cast<const __nv_bfloat16*>(k_idx);
+    const int T = q_begin + rows;  // query rows the tensor map of q_idx covers
+    // windows of at most rw rows that do not straddle the dense / filtered boundary
+    for (long long q0 = q_begin; q0 < T;) {
+        long long q1 = q0 + rw < T ? q0 + rw : T;
+        if (q0 < kDenseRows && q1 > kDenseRows) q1 = kDenseRows;
+        const int nr = (int)(q1 - q0);
+        int* out = idx + (q0 - q_begin) * ld_idx;
+        cudaError_t e;
+        if (q1 <= kDenseRows) {
+            // short rows: dense scores and the dense top-k
+            e = launch_indexer_bf16_prefill(qi, ki, w, T, S, (int)q0, nr, dense, L.ld_dense, cs,
+                                            ctx);
+            if (e == cudaSuccess)
+                e = launch_topk(dense, L.ld_dense, nr, (int)q0, nullptr, (int)q1, k, out, ld_idx,
+                                cs, ctx);
+        } else {
+            // 1. scores of one key tile in 16; 2. per-row thresholds
+            e = launch_indexer_bf16_sample(qi, ki, w, T, S, (int)q0, nr, kSampleStride, sample,
+                                           L.ld_sample, cs, ctx);
+            if (e == cudaSuccess)
+                e = launch_topk_threshold(sample, L.ld_sample, (int)q0, nr, kSampleStride, k, tau,
+                                          fb_any, cs);
+            // 3. every score, keeping only the keys at or above the thresholds
+            if (e == cudaSuccess)
+                e = launch_indexer_bf16_filter(qi, ki, w, T, S, (int)q0, nr, tau, cand, ccount,
+                                               kListCap, (int)L.nchunk_max, cs, ctx);
+            // 4. exact top-k from the candidates
+            if (e == cudaSuccess)
+                e = launch_topk_candidates(cand, ccount, kListCap, (int)L.nchunk_max, (int)q0, nr,
+                                           (int)q1, k, out, ld_idx, fb_row, fb_any, cs);
+            // 5. rows the candidates could not settle: dense scores of the window and the
+            //    dense top-k of those rows (both return at once when no row was flagged)
+            if (e == cudaSuccess)
+                e = launch_indexer_bf16_prefill(qi, ki, w, T, S, (int)q0, nr, dense, L.ld_dense,
+                                                cs, ctx, fb_any);
+            if (e == cudaSuccess)
+                e = launch_topk(dense, L.ld_dense, nr, (int)q0, nullptr, (int)q1, k, out, ld_idx,
+                                cs, ctx, fb_row);
+        }
+        if (e != cudaSuccess) return cuda_fail(e, "index selection launch");
+        q0 = q1;
+    }
+    return DSA_OK;
+}
+
 dsa_status dsa_layer_stack(const char* pattern, int num_layers, int T, int topk, int H_I,
                            int D_I, int H, int D_qk, int D_v, float scale,
                            const void* const* q_idx, const void* const* k_idx,

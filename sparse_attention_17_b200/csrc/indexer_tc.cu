@@ -41,6 +41,7 @@ constexpr int kEpiWarps = 16;      // four per TMEM lane quadrant
 constexpr uint32_t kTileBytes = kBM * 128;  // 128 keys x 64 bf16
 constexpr int kDecodeChunkTiles = 16;       // decode unit = 2048 keys
 constexpr int kPrefillChunkTiles = 32;      // prefill unit: at most 4096 keys
+static_assert(kPrefillChunkTiles * 128 == 4096, "filtered candidate lists are per 4096-key chunk");
 
 template <int QB>
 struct IdxSmem {
@@ -55,10 +56,30 @@ struct IdxSmem {
     int abort;
 };
 
+// What the prefill epilogue does with each score.
+enum IdxMode : int {
+    kDense = 0,    // store every causal score in a dense row
+    kSample = 1,   // scores of every tile_stride-th key tile only, stored compactly
+    kFilter = 2,   // append the keys at or above the row's threshold to candidate lists
+                   // (no dense row)
+};
+
 struct IdxParams {
     const float* w;
     float* scores;
     long long ld;
+    int tile_stride;          // physical key tile of logical tile j = j * tile_stride
+    const int* guard;         // non-null: the launch does nothing unless *guard != 0
+    // kFilter: a row's candidates are kept in one list per (4096-key chunk, TMEM lane
+    // quadrant), so that each list has a single writer (one epilogue warp) and needs no
+    // atomics: list (r, c, q) holds cq slots of {order key, key index} at
+    // cand[((r * nchunk_max + c) * 4 + q) * cq] and its length (also past cq) in
+    // ccount[(r * nchunk_max + c) * 4 + q]
+    const uint32_t* tau;      // per row: threshold as an order key
+    uint2* cand;
+    uint32_t* ccount;
+    int cq, nchunk_max;
+
     int q_begin, q_end;  // prefill query rows [q_begin, q_end)
     int S;               // prefill: key rows
     int num_units;
@@ -94,9 +115,12 @@ struct UnitInfo {
     int len;        // decode: valid keys of the sequence
 };
 
-// Prefill: first query block whose causal key range reaches key chunk c.
-__host__ __device__ __forceinline__ int first_block_of_chunk(int c, int q_begin, int QB) {
-    const long long need = (long long)c * kPrefillChunkTiles * kBM - q_begin - QB + 1;
+// Prefill: first query block whose causal key range reaches key chunk c (chunks count
+// logical tiles, of which each is tile_stride physical tiles apart).
+__host__ __device__ __forceinline__ int first_block_of_chunk(int c, int q_begin, int QB,
+                                                            int tile_stride) {
+    const long long need =
+        (long long)c * kPrefillChunkTiles * kBM * tile_stride - q_begin - QB + 1;
     return need <= 0 ? 0 : (int)((need + QB - 1) / QB);
 }
 
@@ -107,14 +131,14 @@ __device__ __forceinline__ UnitInfo<QB, PAGED> unit_info(const IdxParams& p, int
         // units are enumerated chunk by chunk: chunk c covers blocks first_block(c)..nb-1
         int c = 0, rem = u, b = 0;
         for (; c < p.nchunks; ++c) {
-            const int b0 = min(first_block_of_chunk(c, p.q_begin, QB), p.nb);
+            const int b0 = min(first_block_of_chunk(c, p.q_begin, QB, p.tile_stride), p.nb);
             const int cnt = p.nb - b0;
             if (rem < cnt) { b = b0 + rem; break; }
             rem -= cnt;
         }
         x.row0 = p.q_begin + b * QB;
         const int t_max = min(x.row0 + QB, p.q_end) - 1;
-        const int total = t_max / kBM + 1;
+        const int total = t_max / (kBM * p.tile_stride) + 1;  // logical tiles reaching t_max
         x.tile0 = c * kPrefillChunkTiles;
         x.ntiles = max(0, min(kPrefillChunkTiles, total - x.tile0));
         x.len = min(x.row0 + QB, p.q_end) - x.row0;  // queries in the block
@@ -132,7 +156,7 @@ __device__ __forceinline__ UnitInfo<QB, PAGED> unit_info(const IdxParams& p, int
     return x;
 }
 
-template <int QB, bool PAGED>
+template <int QB, bool PAGED, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                   const __grid_constant__ CUtensorMap tmap_k, const IdxParams p) {
@@ -143,6 +167,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, 0, 0);
     using Smem = IdxSmem<QB>;
 
+    static_assert(MODE == kDense || !PAGED, "decode stores dense rows");
+    if (p.guard != nullptr && *p.guard == 0) return;  // a fallback launch with nothing to do
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5;
@@ -196,7 +222,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 const int st = it % kStages;
                 const uint32_t ph = (it / kStages) & 1;
                 if (!mbar_wait(&sm.k_empty[st], ph ^ 1, abort, p.err)) { ok = false; break; }
-                const int tile = x.tile0 + j;
+                const int tile = (x.tile0 + j) * (PAGED ? 1 : p.tile_stride);
                 if constexpr (!PAGED) {
                     mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
                     tma_load_2d(sm.k[st], &tmap_k, 0, tile * kBM, &sm.k_full[st]);
@@ -263,13 +289,23 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const int qb = ui & 1;
             if (!mbar_wait(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err)) break;
             const float* wbuf = sm.w[qb] + part * QPW * kHI;  // this warp's queries' weights
+            uint32_t tau[QPW];   // kFilter: the thresholds of this warp's queries
+            uint32_t ncand[QPW]; // kFilter: candidates this warp appended per query
+#pragma unroll
+            for (int qi = 0; qi < QPW; ++qi) {
+                const int r = x.row0 + part * QPW + qi - p.q_begin;
+                tau[qi] = (MODE == kFilter && part * QPW + qi < x.len) ? __ldg(p.tau + r) : 0u;
+                ncand[qi] = 0u;
+            }
+            const int chunk = x.tile0 / kPrefillChunkTiles;
             bool ok = true;
             for (int j = 0; j < x.ntiles; ++j, ++it) {
                 const int ab = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
                 if (!mbar_wait(&sm.acc_full[ab], aph, abort, p.err)) { ok = false; break; }
                 tc_fence_after();
-                const int s = (x.tile0 + j) * kBM + quad * 32 + lane;
+                const int lt = x.tile0 + j;  // logical tile
+                const int s = lt * (PAGED ? 1 : p.tile_stride) * kBM + quad * 32 + lane;
                 const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + ab * kAccCols;
                 if (active) {
                     constexpr int QW = QPW < 2 ? QPW : 2;  // queries per TMEM load round
@@ -297,12 +333,35 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                                       fmaxf(__uint_as_float(rv[3]), 0.f));
                             }
                             const float score = acc0 + acc1;
-                            if constexpr (!PAGED) {
+                            if constexpr (PAGED) {
+                                if (s < x.len) p.scores[(long long)x.row0 * p.ld + s] = score;
+                            } else if constexpr (MODE == kDense) {
                                 const int t = x.row0 + qidx;
                                 if (qidx < x.len && s <= t)
                                     p.scores[(long long)(t - p.q_begin) * p.ld + s] = score;
+                            } else if constexpr (MODE == kSample) {
+                                // compact sample row: logical tile lt at columns lt*128..
+                                const int t = x.row0 + qidx;
+                                if (qidx < x.len && s <= t)
+                                    p.scores[(long long)(t - p.q_begin) * p.ld + lt * kBM +
+                                             quad * 32 + lane] = score;
                             } else {
-                                if (s < x.len) p.scores[(long long)x.row0 * p.ld + s] = score;
+                                // the warp's 32 lanes are 32 consecutive keys: one ballot is
+                                // one append batch of the (row, chunk, quadrant) list
+                                const int t = x.row0 + qidx;
+                                const long long r = t - p.q_begin;
+                                const bool valid = qidx < x.len && s <= t;
+                                const uint32_t key = float_order_key(score);
+                                const int qo = qidx - part * QPW;
+                                const bool gt = valid && key >= tau[qo];
+                                const unsigned gtm = __ballot_sync(0xffffffffu, gt);
+                                if (gtm) {
+                                    const uint32_t pos = ncand[qo] + __popc(gtm & ((1u << lane) - 1u));
+                                    if (gt && pos < (uint32_t)p.cq)
+                                        p.cand[((r * p.nchunk_max + chunk) * 4 + quad) * p.cq + pos] =
+                                            make_uint2(key, (uint32_t)s);
+                                    ncand[qo] += __popc(gtm);
+                                }
                             }
                         }
                     }
@@ -312,6 +371,15 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                 if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
             }
             if (!ok) break;
+            if constexpr (MODE == kFilter) {
+                if (active && lane < QPW && part * QPW + lane < x.len) {
+                    uint32_t nc = 0;
+#pragma unroll
+                    for (int qi = 0; qi < QPW; ++qi) nc = lane == qi ? ncand[qi] : nc;
+                    const long long r = x.row0 + part * QPW + lane - p.q_begin;
+                    p.ccount[(r * p.nchunk_max + chunk) * 4 + quad] = nc;
+                }
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.q_empty[qb]);  // done with this unit's weights
         }
@@ -330,16 +398,46 @@ size_t indexer_smem_bytes() {
     return sizeof(IdxSmem<QB>) + 1024;
 }
 
-template <int QB, bool PAGED>
+template <int QB, bool PAGED, int MODE>
 cudaError_t launch_indexer_tc(const CUtensorMap& tq, const CUtensorMap& tk, const IdxParams& p,
                               int grid, cudaStream_t stream) {
     const size_t smem = indexer_smem_bytes<QB, PAGED>();
-    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<QB, PAGED>,
+    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<QB, PAGED, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    indexer_tc_kernel<QB, PAGED><<<grid, kThreads, smem, stream>>>(tq, tk, p);
+    indexer_tc_kernel<QB, PAGED, MODE><<<grid, kThreads, smem, stream>>>(tq, tk, p);
     count_launch(DSA_KERNEL_INDEXER);
     return cudaGetLastError();
+}
+
+// Prefill launch of any mode: tensor maps, the unit count of the window and the grid.
+template <int MODE>
+cudaError_t launch_prefill(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_idx, int T, int S,
+                           IdxParams p, cudaStream_t stream, const DevCtx& ctx) {
+    constexpr int QB = 16;
+    CUtensorMap tq, tk;
+    if (!make_tmap_bf16_2d(&tq, q_idx, (uint64_t)T * kHI, kDI, kDI * 2, QB * kHI, kDI))
+        return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tk, k_idx, (uint64_t)S, kDI, kDI * 2, kBM, kDI))
+        return cudaErrorInvalidValue;
+    const int rows = p.q_end - p.q_begin;
+    p.S = S;
+    p.nb = (rows + QB - 1) / QB;
+    {
+        const int t_max = p.q_end - 1;
+        const int logical_tiles = t_max / (kBM * p.tile_stride) + 1;
+        p.nchunks = (logical_tiles + kPrefillChunkTiles - 1) / kPrefillChunkTiles;
+        long long units = 0;
+        for (int c = 0; c < p.nchunks; ++c) {
+            int b0 = first_block_of_chunk(c, p.q_begin, QB, p.tile_stride);
+            units += p.nb - (b0 < p.nb ? b0 : p.nb);
+        }
+        p.num_units = (int)units;
+    }
+    p.err = ctx.err;
+    const int grid = p.num_units < ctx.num_sms ? p.num_units : ctx.num_sms;
+    if (grid <= 0) return cudaSuccess;
+    return launch_indexer_tc<QB, false, MODE>(tq, tk, p, grid, stream);
 }
 
 }  // namespace
@@ -347,34 +445,47 @@ cudaError_t launch_indexer_tc(const CUtensorMap& tq, const CUtensorMap& tk, cons
 cudaError_t launch_indexer_bf16_prefill(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_idx,
                                         const float* w, int T, int S, int q_begin, int rows,
                                         float* scores, long long ld, cudaStream_t stream,
-                                        const DevCtx& ctx) {
-    constexpr int QB = 16;
-    CUtensorMap tq, tk;
-    if (!make_tmap_bf16_2d(&tq, q_idx, (uint64_t)T * kHI, kDI, kDI * 2, QB * kHI, kDI))
-        return cudaErrorInvalidValue;
-    if (!make_tmap_bf16_2d(&tk, k_idx, (uint64_t)S, kDI, kDI * 2, kBM, kDI))
-        return cudaErrorInvalidValue;
+                                        const DevCtx& ctx, const int* guard) {
     IdxParams p{};
     p.w = w;
     p.scores = scores;
     p.ld = ld;
+    p.tile_stride = 1;
+    p.guard = guard;
     p.q_begin = q_begin;
     p.q_end = q_begin + rows;
-    p.S = S;
-    p.nb = (rows + QB - 1) / QB;
-    {
-        const int t_max = q_begin + rows - 1;
-        p.nchunks = (t_max / kBM + 1 + kPrefillChunkTiles - 1) / kPrefillChunkTiles;
-        long long units = 0;
-        for (int c = 0; c < p.nchunks; ++c) {
-            int b0 = first_block_of_chunk(c, q_begin, QB);
-            units += p.nb - (b0 < p.nb ? b0 : p.nb);
-        }
-        p.num_units = (int)units;
-    }
-    p.err = ctx.err;
-    const int grid = p.num_units < ctx.num_sms ? p.num_units : ctx.num_sms;
-    return launch_indexer_tc<QB, false>(tq, tk, p, grid, stream);
+    return launch_prefill<kDense>(q_idx, k_idx, T, S, p, stream, ctx);
+}
+
+cudaError_t launch_indexer_bf16_sample(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_idx,
+                                       const float* w, int T, int S, int q_begin, int rows,
+                                       int tile_stride, float* sample, long long ld_sample,
+                                       cudaStream_t stream, const DevCtx& ctx) {
+    IdxParams p{};
+    p.w = w;
+    p.scores = sample;
+    p.ld = ld_sample;
+    p.tile_stride = tile_stride;
+    p.q_begin = q_begin;
+    p.q_end = q_begin + rows;
+    return launch_prefill<kSample>(q_idx, k_idx, T, S, p, stream, ctx);
+}
+
+cudaError_t launch_indexer_bf16_filter(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_idx,
+                                       const float* w, int T, int S, int q_begin, int rows,
+                                       const uint32_t* tau, uint2* cand, uint32_t* ccount, int cq,
+                                       int nchunk_max, cudaStream_t stream, const DevCtx& ctx) {
+    IdxParams p{};
+    p.w = w;
+    p.tile_stride = 1;
+    p.tau = tau;
+    p.cand = cand;
+    p.ccount = ccount;
+    p.cq = cq;
+    p.nchunk_max = nchunk_max;
+    p.q_begin = q_begin;
+    p.q_end = q_begin + rows;
+    return launch_prefill<kFilter>(q_idx, k_idx, T, S, p, stream, ctx);
 }
 
 cudaError_t launch_indexer_bf16_decode(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_pool,
@@ -401,7 +512,8 @@ cudaError_t launch_indexer_bf16_decode(const __nv_bfloat16* q_idx, const __nv_bf
     p.num_units = B * units_per_seq;
     p.err = ctx.err;
     const int grid = p.num_units < ctx.num_sms ? p.num_units : ctx.num_sms;
-    return launch_indexer_tc<1, true>(tq, tk, p, grid, stream);
+    p.tile_stride = 1;
+    return launch_indexer_tc<1, true, kDense>(tq, tk, p, grid, stream);
 }
 
 }  // namespace dsa

@@ -33,10 +33,28 @@ cudaError_t launch_indexer_f32(const float* q_idx, const float* k_idx, const flo
                                int D_I, int q_begin, int rows, float* scores, long long ld,
                                cudaStream_t stream);
 
+// Dense prefill scores of query rows [q_begin, q_begin+rows).  With `guard` non-null the
+// launch does nothing unless *guard != 0 (the filtered path's fallback).
 cudaError_t launch_indexer_bf16_prefill(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_idx,
                                         const float* w, int T, int S, int q_begin, int rows,
                                         float* scores, long long ld, cudaStream_t stream,
-                                        const DevCtx& ctx);
+                                        const DevCtx& ctx, const int* guard = nullptr);
+
+// Scores of every tile_stride-th 128-key tile only, stored compactly: row r, logical tile j
+// at sample[r * ld_sample + j * 128 ...] (causal entries only).
+cudaError_t launch_indexer_bf16_sample(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_idx,
+                                       const float* w, int T, int S, int q_begin, int rows,
+                                       int tile_stride, float* sample, long long ld_sample,
+                                       cudaStream_t stream, const DevCtx& ctx);
+
+// Filtered prefill scores: for row r, every causal key with order key >= tau[r] is
+// appended to the list of its 4096-key chunk c and TMEM lane quadrant q (the key's bits
+// 5..6): cand[((r * nchunk_max + c) * 4 + q) * cq ..] ({order key, key index}) with its
+// length in ccount[(r * nchunk_max + c) * 4 + q] (also when past cq).
+cudaError_t launch_indexer_bf16_filter(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_idx,
+                                       const float* w, int T, int S, int q_begin, int rows,
+                                       const uint32_t* tau, uint2* cand, uint32_t* ccount, int cq,
+                                       int nchunk_max, cudaStream_t stream, const DevCtx& ctx);
 
 cudaError_t launch_indexer_bf16_decode(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_pool,
                                        const float* w, int B, long long pool_rows,
@@ -44,9 +62,26 @@ cudaError_t launch_indexer_bf16_decode(const __nv_bfloat16* q_idx, const __nv_bf
                                        const int* seq_lens, int max_len, float* scores,
                                        long long ld, cudaStream_t stream, const DevCtx& ctx);
 
+// Per-row top-k of dense score rows.  With row_mask non-null, only rows r with
+// row_mask[r] != 0 are processed (the filtered path's fallback).
 cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin,
                         const int* row_len, int max_len, int k, int* idx, long long ld_idx,
-                        cudaStream_t stream, const DevCtx& ctx);
+                        cudaStream_t stream, const DevCtx& ctx, const int* row_mask = nullptr);
+
+// Filtered path, step 2: per-row threshold tau (an order key) from the compact sampled
+// scores of launch_indexer_bf16_sample.  Clears *fb_any.
+cudaError_t launch_topk_threshold(const float* sample, long long ld_sample, int q_begin, int rows,
+                                  int tile_stride, int k, uint32_t* tau, int* fb_any,
+                                  cudaStream_t stream);
+
+// Filtered path, step 4: exact top-k of each row from its candidate lists (the output of
+// launch_indexer_bf16_filter).  Rows it cannot settle (a list past cq, more candidates than
+// the selection buffer holds, or fewer than k) get fb_row[r] = 1 and *fb_any = 1 and are
+// left for the dense fallback.
+cudaError_t launch_topk_candidates(const uint2* cand, const uint32_t* ccount, int cq,
+                                   int nchunk_max, int q_begin, int rows, int max_len, int k,
+                                   int* idx, long long ld_idx, int* fb_row, int* fb_any,
+                                   cudaStream_t stream);
 
 cudaError_t launch_sparse_mha_f32(const float* q, const float* k, const float* v, int num_q,
                                   int H, int D, float scale, long long kv_rows, const int* idx,

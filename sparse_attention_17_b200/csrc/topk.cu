@@ -36,6 +36,7 @@ constexpr int kCandCap = 8192;
 constexpr int kStride = kWarps * 32;  // elements covered by all warps per iteration
 constexpr int kSlice = kCandCap / kWarps;  // candidate entries owned by one warp
 constexpr int kUnroll = 4;                 // 16-byte loads in flight per thread
+constexpr int kBM_SAMPLE = 128;            // keys per sampled tile (the indexer's tile)
 
 struct TopkScratch {
     uint32_t hist[kBins];
@@ -304,10 +305,54 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
     return need;
 }
 
+// Keeps the first `need` ties (tie bitmap) in index order, merges them into the selection
+// bitmap and writes the selected key positions in ascending order, then -1 up to k.
+__device__ void trim_ties_and_compact(TopkScratch& sh, uint32_t* sel, const uint32_t* tie,
+                                      int nwords, uint32_t need, int k, int* out) {
+    const int wpt = (nwords + kThreads - 1) / kThreads;
+    const int w0 = threadIdx.x * wpt;
+    const int w1 = min(w0 + wpt, nwords);
+    uint32_t local = 0;
+    for (int w = w0; w < w1; ++w) local += __popc(tie[w]);
+    uint32_t total;
+    uint32_t before = block_exclusive_scan(local, sh, &total);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t tb = tie[w];
+        const uint32_t c = __popc(tb);
+        if (before >= need) {
+            tb = 0u;
+        } else if (before + c > need) {
+            uint32_t keep = 0u, rest = tb;
+            for (uint32_t m = need - before; m > 0; --m) {
+                keep |= rest & (0u - rest);
+                rest &= rest - 1u;
+            }
+            tb = keep;
+        }
+        before += c;
+        sel[w] |= tb;
+    }
+    __syncthreads();
+    local = 0;
+    for (int w = w0; w < w1; ++w) local += __popc(sel[w]);
+    uint32_t pos = block_exclusive_scan(local, sh, &total);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t bits = sel[w];
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1u;
+            if (pos < (uint32_t)k) out[pos] = w * 32 + b;
+            ++pos;
+        }
+    }
+    for (int i = (int)total + threadIdx.x; i < k; i += kThreads) out[i] = -1;
+}
+
 __global__ void __launch_bounds__(kThreads, 2)
 topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
                   const int* __restrict__ row_len, int max_len, int k, int* __restrict__ idx,
-                  long long ld_idx, unsigned* __restrict__ err) {
+                  long long ld_idx, const int* __restrict__ row_mask, unsigned* __restrict__ err) {
+    if (row_mask != nullptr && row_mask[blockIdx.x] == 0) return;  // row not asked for
     extern __shared__ __align__(16) unsigned char smem_raw[];
     TopkScratch& sh = *reinterpret_cast<TopkScratch*>(smem_raw);
     uint32_t* sel = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkScratch));
@@ -434,46 +479,190 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
     }
     __syncthreads();
 
-    // ---- keep the first `need` ties in index order, merge, compact ascending ----
-    const int wpt = (nwords + kThreads - 1) / kThreads;
-    const int w0 = threadIdx.x * wpt;
-    const int w1 = min(w0 + wpt, nwords);
-    uint32_t local = 0;
-    for (int w = w0; w < w1; ++w) local += __popc(tie[w]);
-    uint32_t total;
-    uint32_t before = block_exclusive_scan(local, sh, &total);
-    for (int w = w0; w < w1; ++w) {
-        uint32_t tb = tie[w];
-        const uint32_t c = __popc(tb);
-        if (before >= need) {
-            tb = 0u;
-        } else if (before + c > need) {
-            uint32_t keep = 0u, rest = tb;
-            for (uint32_t m = need - before; m > 0; --m) {
-                keep |= rest & (0u - rest);
-                rest &= rest - 1u;
-            }
-            tb = keep;
-        }
-        before += c;
-        sel[w] |= tb;
-    }
-    __syncthreads();
-    local = 0;
-    for (int w = w0; w < w1; ++w) local += __popc(sel[w]);
-    uint32_t pos = block_exclusive_scan(local, sh, &total);
-    for (int w = w0; w < w1; ++w) {
-        uint32_t bits = sel[w];
-        while (bits) {
-            const int b = __ffs(bits) - 1;
-            bits &= bits - 1u;
-            if (pos < (uint32_t)k) out[pos] = w * 32 + b;
-            ++pos;
-        }
-    }
-    for (int i = (int)total + threadIdx.x; i < k; i += kThreads) out[i] = -1;
+    trim_ties_and_compact(sh, sel, tie, nwords, need, k, out);
 }
 
+
+// ---------------------------------------------------------------------------------------
+// Filtered selection (no dense score rows): thresholds from sampled scores, then the exact
+// top-k among the candidates the filtered indexer appended.
+// ---------------------------------------------------------------------------------------
+constexpr int kThrWarps = 4;          // rows per threshold CTA (one warp each)
+constexpr int kThrBins = 2048;        // 11-bit digits
+
+// Warp-level: the bin b (counting from the top) where above(b) < need <= above(b)+hist[b].
+__device__ __forceinline__ void warp_find_bin(const uint32_t* hist, uint32_t need,
+                                              uint32_t* bin, uint32_t* above_out) {
+    const int lane = threadIdx.x & 31;
+    constexpr int per = kThrBins / 32;
+    const int top = kThrBins - 1 - lane * per;  // this lane's highest bin
+    uint32_t local = 0;
+    for (int i = 0; i < per; ++i) local += hist[top - i];
+    uint32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const uint32_t above = incl - local;
+    const unsigned owner = __ballot_sync(0xffffffffu, above < need && incl >= need);
+    const int src = owner ? __ffs(owner) - 1 : 31;
+    uint32_t b = 0, ab = 0;
+    if (lane == src) {
+        uint32_t acc = above;
+        b = (uint32_t)(top - per + 1);
+        for (int i = 0; i < per; ++i) {
+            const uint32_t c = hist[top - i];
+            if (acc + c >= need) { b = (uint32_t)(top - i); break; }
+            acc += c;
+        }
+        ab = acc;
+    }
+    *bin = __shfl_sync(0xffffffffu, b, src);
+    *above_out = __shfl_sync(0xffffffffu, ab, src);
+}
+
+// One warp per row: tau[r] = a lower bound of the rank-th largest sampled score (the lower
+// edge of its 22-bit bin), rank = e + 6 sqrt(e) + 2 for the e = k * m / n samples expected
+// above the row's k-th largest score.  The first CTA also clears the window's fallback
+// flag.  Samples are read 16 per lane at a time, all in flight together.
+constexpr int kThrBatch = 16;
+
+__device__ __forceinline__ void threshold_pass(const float* row, int ncols, int span, int t,
+                                               uint32_t* hist, int round, uint32_t b1) {
+    const int lane = threadIdx.x & 31;
+    for (int c0 = 0; c0 < ncols; c0 += 32 * kThrBatch) {
+        float v[kThrBatch];
+#pragma unroll
+        for (int i = 0; i < kThrBatch; ++i) {
+            const int c = c0 + i * 32 + lane;
+            const bool in = c < ncols && (c / kBM_SAMPLE) * span + (c % kBM_SAMPLE) <= t;
+            v[i] = in ? __ldg(row + c) : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < kThrBatch; ++i) {
+            const int c = c0 + i * 32 + lane;
+            const bool in = c < ncols && (c / kBM_SAMPLE) * span + (c % kBM_SAMPLE) <= t;
+            const uint32_t key = float_order_key(v[i]);
+            if (round == 0) hist_add(hist, key >> 21, in);
+            else hist_add(hist, (key >> 10) & 0x7FFu, in && (key >> 21) == b1);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(32 * kThrWarps)
+topk_threshold_kernel(const float* __restrict__ sample, long long ld_sample, int q_begin,
+                      int rows, int tile_stride, int k, uint32_t* __restrict__ tau,
+                      int* __restrict__ fb_any) {
+    __shared__ uint32_t hist_all[kThrWarps][kThrBins];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *fb_any = 0;
+    const int r = blockIdx.x * kThrWarps + warp;
+    if (r >= rows) return;
+    uint32_t* hist = hist_all[warp];
+    const int t = q_begin + r;
+    const int n = t + 1;
+    // valid samples: logical tile j holds keys j*stride*128 .. +127, causal ones only
+    const int span = kBM_SAMPLE * tile_stride;
+    const int ntiles = t / span + 1;
+    const int ncols = ntiles * kBM_SAMPLE;
+    const int m = (ntiles - 1) * kBM_SAMPLE + min(kBM_SAMPLE, n - (ntiles - 1) * span);
+    const float e = (float)k * (float)m / (float)n;
+    uint32_t rank = (uint32_t)ceilf(e + 6.f * sqrtf(e)) + 2u;
+    if (rank > (uint32_t)m) rank = (uint32_t)m;
+    const float* row = sample + (long long)r * ld_sample;
+    for (int i = lane; i < kThrBins; i += 32) hist[i] = 0u;
+    __syncwarp();
+    threshold_pass(row, ncols, span, t, hist, 0, 0u);  // bits 31..21
+    __syncwarp();
+    uint32_t b1, above;
+    warp_find_bin(hist, rank, &b1, &above);
+    const uint32_t need2 = rank - above;
+    __syncwarp();
+    for (int i = lane; i < kThrBins; i += 32) hist[i] = 0u;
+    __syncwarp();
+    threshold_pass(row, ncols, span, t, hist, 1, b1);  // bits 20..10 within bin b1
+    __syncwarp();
+    uint32_t b2, above2;
+    warp_find_bin(hist, need2, &b2, &above2);
+    if (lane == 0) tau[r] = (b1 << 21) | (b2 << 10);
+}
+
+// One CTA per row: the exact top-k among the row's candidates (all keys at or above
+// tau[r], kept in lists per 4096-key chunk and lane quadrant): with at least k of them the
+// k-th largest key and every key equal to it are among them.  Rows whose lists overflowed
+// or with fewer than k candidates are flagged for the dense fallback (fb_row[r] = 1,
+// *fb_any = 1) and left unwritten.
+__global__ void __launch_bounds__(kThreads, 2)
+topk_candidates_kernel(const uint2* __restrict__ cand, const uint32_t* __restrict__ ccount,
+                       int cq, int nchunk_max, int q_begin, int max_len, int k,
+                       int* __restrict__ idx, long long ld_idx, int* __restrict__ fb_row,
+                       int* __restrict__ fb_any) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    TopkScratch& sh = *reinterpret_cast<TopkScratch*>(smem_raw);
+    uint32_t* sel = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkScratch));
+    const int max_words = (max_len + 31) >> 5;
+    uint32_t* tie = sel + max_words;
+
+    const int r = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n = q_begin + r + 1;
+    int* out = idx + (long long)r * ld_idx;
+    if (n <= k) {  // every valid key is selected
+        if (threadIdx.x == 0) fb_row[r] = 0;
+        for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    const int nwords = (n + 31) >> 5;
+    for (int i = threadIdx.x; i < nwords; i += kThreads) sel[i] = 0u;
+    // the row's lists (chunk, quadrant) are dealt round-robin to the warps, each appending
+    // into its slice of the candidate buffer
+    const int nlists = ((n + 4095) >> 12) * 4;
+    const uint32_t* crow = ccount + (long long)r * nchunk_max * 4;
+    const uint2* lrow = cand + (long long)r * nchunk_max * 4 * cq;
+    uint32_t filled = 0;
+    bool over = false;
+    for (int l = warp; l < nlists; l += kWarps) {
+        const uint32_t len = __ldg(crow + l);
+        if (len > (uint32_t)cq || filled + len > (uint32_t)kSlice) { over = true; break; }
+        const uint2* src = lrow + (long long)l * cq;
+        for (uint32_t i = lane; i < len; i += 32) {
+            const uint2 v = __ldg(src + i);
+            sh.cand_key[warp * kSlice + filled + i] = v.x;
+            sh.cand_idx[warp * kSlice + filled + i] = (int)v.y;
+        }
+        filled += len;
+    }
+    if (lane == 0) sh.wcount[warp] = over ? 0xFFFFFFFFu : filled;
+    __syncthreads();
+    uint32_t c = 0;
+    bool fail = false;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        const uint32_t v = sh.wcount[w];
+        fail |= v == 0xFFFFFFFFu;
+        c += v;
+    }
+    if (fail || c < (uint32_t)k) {
+        if (threadIdx.x == 0) { fb_row[r] = 1; atomicExch(fb_any, 1); }
+        return;
+    }
+    for (int i = threadIdx.x; i < nwords; i += kThreads) tie[i] = 0u;
+    uint32_t need;
+    const uint32_t tau = slice_radix_select(sh, (uint32_t)k, true, &need);
+    {
+        const int lo = warp * kSlice, cnt = (int)sh.wcount[warp];
+        for (int i = lane; i < cnt; i += 32) {
+            const uint32_t key = sh.cand_key[lo + i];
+            const int s = sh.cand_idx[lo + i];
+            if (key > tau) atomicOr(&sel[s >> 5], 1u << (s & 31));
+            else if (key == tau) atomicOr(&tie[s >> 5], 1u << (s & 31));
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) fb_row[r] = 0;
+    trim_ties_and_compact(sh, sel, tie, nwords, need, k, out);
+}
 }  // namespace
 
 size_t topk_smem_bytes(int max_len) {
@@ -483,13 +672,38 @@ size_t topk_smem_bytes(int max_len) {
 
 cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin,
                         const int* row_len, int max_len, int k, int* idx, long long ld_idx,
-                        cudaStream_t stream, const DevCtx& ctx) {
+                        cudaStream_t stream, const DevCtx& ctx, const int* row_mask) {
     const size_t smem = topk_smem_bytes(max_len);
     cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     topk_radix_kernel<<<rows, kThreads, smem, stream>>>(scores, ld, q_begin, row_len, max_len, k,
-                                                        idx, ld_idx, ctx.err);
+                                                        idx, ld_idx, row_mask, ctx.err);
+    count_launch(DSA_KERNEL_TOPK);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk_threshold(const float* sample, long long ld_sample, int q_begin, int rows,
+                                  int tile_stride, int k, uint32_t* tau, int* fb_any,
+                                  cudaStream_t stream) {
+    const int grid = (rows + kThrWarps - 1) / kThrWarps;
+    topk_threshold_kernel<<<grid, 32 * kThrWarps, 0, stream>>>(sample, ld_sample, q_begin, rows,
+                                                                tile_stride, k, tau, fb_any);
+    count_launch(DSA_KERNEL_TOPK);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk_candidates(const uint2* cand, const uint32_t* ccount, int cq,
+                                   int nchunk_max, int q_begin, int rows, int max_len, int k,
+                                   int* idx, long long ld_idx, int* fb_row, int* fb_any,
+                                   cudaStream_t stream) {
+    const size_t smem = topk_smem_bytes(max_len);
+    cudaError_t e = cudaFuncSetAttribute(topk_candidates_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topk_candidates_kernel<<<rows, kThreads, smem, stream>>>(cand, ccount, cq, nchunk_max,
+                                                             q_begin, max_len, k, idx, ld_idx,
+                                                             fb_row, fb_any);
     count_launch(DSA_KERNEL_TOPK);
     return cudaGetLastError();
 }

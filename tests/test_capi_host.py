@@ -144,3 +144,24 @@ def test_launch_counters_reset(lib):
     for k in range(4):
         assert dsa.launch_count(k) == 0
     assert dsa.launch_count(9) == -1
+
+
+def test_index_select_rejects_and_sizes(lib):
+    f = lib.dsa_index_select
+    # null tensors, unsupported shapes, bad k / ld_idx, keys beyond S: refused before any launch
+    assert f(None, 16, 16, 16, 64, 0, 8, 64, 8, 16, 8, 256, 1 << 20, None) == _lib.DSA_ERR_INVALID_ARG
+    assert f(16, 16, 16, 2, 16, 0, 8, 64, 8, 16, 8, 256, 1 << 20, None) == _lib.DSA_ERR_UNSUPPORTED
+    assert f(16, 16, 16, 16, 64, 0, 8, 64, 0, 16, 8, 256, 1 << 20, None) == _lib.DSA_ERR_UNSUPPORTED
+    assert f(16, 16, 16, 16, 64, 0, 8, 64, 8, 16, 6, 256, 1 << 20, None) == _lib.DSA_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 64, 60, 8, 64, 8, 16, 8, 256, 1 << 20, None) == _lib.DSA_ERR_INVALID_ARG
+    # workspace: null / misaligned refused; too small for 16 rows refused
+    assert f(16, 16, 16, 16, 64, 0, 64, 64, 8, 16, 8, None, 1 << 20, None) == _lib.DSA_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 64, 0, 64, 64, 8, 16, 8, 272, 1 << 30, None) == _lib.DSA_ERR_INVALID_ARG
+    small = lib.dsa_index_select_workspace_size(8, 65536)
+    assert f(16, 16, 16, 16, 64, 0, 4096, 65536, 8, 16, 8, 256, small, None) == _lib.DSA_ERR_WORKSPACE
+    # zero rows is a no-op
+    assert f(16, 16, 16, 16, 64, 0, 0, 64, 8, 16, 8, 256, 1 << 20, None) == _lib.DSA_OK
+    # the scratch grows with the window and the key count
+    a = lib.dsa_index_select_workspace_size(16, 8192)
+    assert 0 < a < lib.dsa_index_select_workspace_size(32, 8192) < lib.dsa_index_select_workspace_size(32, 65536)
+    assert lib.dsa_index_select_workspace_size(0, 8192) == 0
