@@ -305,7 +305,9 @@ def run_native(args, rank, world, local_rank):
         out_host = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
         d2h = out_host[0].numel() * out_host[0].element_size()
         s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        n_e2e = max(2, min(args.steps, 6))
+        # as many steps as the device-timed run: the first upload and the last download
+        # (pipeline fill and drain) are part of the measurement, spread over the K steps
+        n_e2e = max(2, args.steps)
 
         def e2e_run(n):
             ev_up = [torch.cuda.Event() for _ in range(n)]

@@ -2,6 +2,7 @@
 //
 // Every entry point validates its arguments on the host and returns before launching
 // anything when they are wrong; then it calls the launchers of the kernel files.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -326,11 +327,11 @@ size_t dsa_layer_stack_workspace_size(int T, int rows_window) {
 // ---- filtered index selection (dsa_index_select) ----
 namespace {
 
-constexpr int kSampleStride = 16;     // one 128-key tile in 16 is scored for the thresholds
 constexpr int kDenseRows = 8192;      // rows with at most this many keys take the dense path
 constexpr int kListCap = 512;         // candidates per (row, 4096-key chunk, lane quadrant)
 
 struct SelectLayout {
+    int sample_stride;  // one 128-key tile in sample_stride is scored for the thresholds
     long long ld_sample, ld_dense, nchunk_max;
     size_t off_sample, off_tau, off_fb_row, off_fb_any, off_ccount, off_cand, off_dense;
     size_t total;
@@ -340,8 +341,12 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 SelectLayout select_layout(long long rows, long long S) {
     SelectLayout L{};
-    const long long span = 128LL * kSampleStride;
-    L.ld_sample = (S + span - 1) / span * 128;
+    // at most topk_sample_max() sampled keys per row: a stride of at least 16 tiles, more
+    // for long rows
+    const long long tiles = (S + 127) / 128;
+    const long long max_tiles = topk_sample_max() / 128;
+    L.sample_stride = (int)std::max(16LL, (tiles + max_tiles - 1) / max_tiles);
+    L.ld_sample = topk_sample_max();
     L.ld_dense = (S + 3) / 4 * 4;
     L.nchunk_max = (S + 4095) / 4096;
     const long long lists = rows * L.nchunk_max * 4;
@@ -424,12 +429,12 @@ dsa_status dsa_index_select(const void* q_idx, const void* k_idx, const float* w
                 e = launch_topk(dense, L.ld_dense, nr, (int)q0, nullptr, (int)q1, k, out, ld_idx,
                                 cs, ctx);
         } else {
-            // 1. scores of one key tile in 16; 2. per-row thresholds
-            e = launch_indexer_bf16_sample(qi, ki, w, T, S, (int)q0, nr, kSampleStride, sample,
+            // 1. scores of one key tile in sample_stride; 2. per-row thresholds
+            e = launch_indexer_bf16_sample(qi, ki, w, T, S, (int)q0, nr, L.sample_stride, sample,
                                            L.ld_sample, cs, ctx);
             if (e == cudaSuccess)
-                e = launch_topk_threshold(sample, L.ld_sample, (int)q0, nr, kSampleStride, k, tau,
-                                          fb_any, cs);
+                e = launch_topk_threshold(sample, L.ld_sample, (int)q0, nr, L.sample_stride, k,
+                                          tau, fb_any, cs);
             // 3. every score, keeping only the keys at or above the thresholds
             if (e == cudaSuccess)
                 e = launch_indexer_bf16_filter(qi, ki, w, T, S, (int)q0, nr, tau, cand, ccount,

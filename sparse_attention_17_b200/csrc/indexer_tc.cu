@@ -289,12 +289,15 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const int qb = ui & 1;
             if (!mbar_wait(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err)) break;
             const float* wbuf = sm.w[qb] + part * QPW * kHI;  // this warp's queries' weights
-            uint32_t tau[QPW];   // kFilter: the thresholds of this warp's queries
+            float tau[QPW];      // kFilter: the thresholds of this warp's queries as floats
             uint32_t ncand[QPW]; // kFilter: candidates this warp appended per query
 #pragma unroll
             for (int qi = 0; qi < QPW; ++qi) {
                 const int r = x.row0 + part * QPW + qi - p.q_begin;
-                tau[qi] = (MODE == kFilter && part * QPW + qi < x.len) ? __ldg(p.tau + r) : 0u;
+                // an order key >= tau[r] is exactly a score >= the float the key stands for
+                const uint32_t tk =
+                    (MODE == kFilter && part * QPW + qi < x.len) ? __ldg(p.tau + r) : 0u;
+                tau[qi] = __uint_as_float((tk & 0x80000000u) ? (tk & 0x7FFFFFFFu) : ~tk);
                 ncand[qi] = 0u;
             }
             const int chunk = x.tile0 / kPrefillChunkTiles;
@@ -351,15 +354,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                                 const int t = x.row0 + qidx;
                                 const long long r = t - p.q_begin;
                                 const bool valid = qidx < x.len && s <= t;
-                                const uint32_t key = float_order_key(score);
                                 const int qo = qidx - part * QPW;
-                                const bool gt = valid && key >= tau[qo];
+                                const bool gt = valid && score >= tau[qo];
                                 const unsigned gtm = __ballot_sync(0xffffffffu, gt);
                                 if (gtm) {
                                     const uint32_t pos = ncand[qo] + __popc(gtm & ((1u << lane) - 1u));
                                     if (gt && pos < (uint32_t)p.cq)
                                         p.cand[((r * p.nchunk_max + chunk) * 4 + quad) * p.cq + pos] =
-                                            make_uint2(key, (uint32_t)s);
+                                            make_uint2(float_order_key(score), (uint32_t)s);
                                     ncand[qo] += __popc(gtm);
                                 }
                             }

@@ -68,8 +68,12 @@ cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin
                         const int* row_len, int max_len, int k, int* idx, long long ld_idx,
                         cudaStream_t stream, const DevCtx& ctx, const int* row_mask = nullptr);
 
+// Sampled keys per row the threshold kernel holds at most (tiles x 128).
+int topk_sample_max();
+
 // Filtered path, step 2: per-row threshold tau (an order key) from the compact sampled
-// scores of launch_indexer_bf16_sample.  Clears *fb_any.
+// scores of launch_indexer_bf16_sample (at most topk_sample_max() per row).  Clears
+// *fb_any.
 cudaError_t launch_topk_threshold(const float* sample, long long ld_sample, int q_begin, int rows,
                                   int tile_stride, int k, uint32_t* tau, int* fb_any,
                                   cudaStream_t stream);

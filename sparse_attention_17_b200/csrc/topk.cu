@@ -487,79 +487,29 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
 // Filtered selection (no dense score rows): thresholds from sampled scores, then the exact
 // top-k among the candidates the filtered indexer appended.
 // ---------------------------------------------------------------------------------------
-constexpr int kThrWarps = 4;          // rows per threshold CTA (one warp each)
-constexpr int kThrBins = 2048;        // 11-bit digits
+constexpr int kRowWarps = 8;          // rows per CTA of the warp-per-row kernels
+constexpr int kSampleMax = 2048;      // sampled keys per row at most (64 per lane)
 
-// Warp-level: the bin b (counting from the top) where above(b) < need <= above(b)+hist[b].
-__device__ __forceinline__ void warp_find_bin(const uint32_t* hist, uint32_t need,
-                                              uint32_t* bin, uint32_t* above_out) {
-    const int lane = threadIdx.x & 31;
-    constexpr int per = kThrBins / 32;
-    const int top = kThrBins - 1 - lane * per;  // this lane's highest bin
-    uint32_t local = 0;
-    for (int i = 0; i < per; ++i) local += hist[top - i];
-    uint32_t incl = local;
+__device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    const uint32_t above = incl - local;
-    const unsigned owner = __ballot_sync(0xffffffffu, above < need && incl >= need);
-    const int src = owner ? __ffs(owner) - 1 : 31;
-    uint32_t b = 0, ab = 0;
-    if (lane == src) {
-        uint32_t acc = above;
-        b = (uint32_t)(top - per + 1);
-        for (int i = 0; i < per; ++i) {
-            const uint32_t c = hist[top - i];
-            if (acc + c >= need) { b = (uint32_t)(top - i); break; }
-            acc += c;
-        }
-        ab = acc;
-    }
-    *bin = __shfl_sync(0xffffffffu, b, src);
-    *above_out = __shfl_sync(0xffffffffu, ab, src);
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
 }
 
-// One warp per row: tau[r] = a lower bound of the rank-th largest sampled score (the lower
-// edge of its 22-bit bin), rank = e + 6 sqrt(e) + 2 for the e = k * m / n samples expected
-// above the row's k-th largest score.  The first CTA also clears the window's fallback
-// flag.  Samples are read 16 per lane at a time, all in flight together.
-constexpr int kThrBatch = 16;
-
-__device__ __forceinline__ void threshold_pass(const float* row, int ncols, int span, int t,
-                                               uint32_t* hist, int round, uint32_t b1) {
-    const int lane = threadIdx.x & 31;
-    for (int c0 = 0; c0 < ncols; c0 += 32 * kThrBatch) {
-        float v[kThrBatch];
-#pragma unroll
-        for (int i = 0; i < kThrBatch; ++i) {
-            const int c = c0 + i * 32 + lane;
-            const bool in = c < ncols && (c / kBM_SAMPLE) * span + (c % kBM_SAMPLE) <= t;
-            v[i] = in ? __ldg(row + c) : 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < kThrBatch; ++i) {
-            const int c = c0 + i * 32 + lane;
-            const bool in = c < ncols && (c / kBM_SAMPLE) * span + (c % kBM_SAMPLE) <= t;
-            const uint32_t key = float_order_key(v[i]);
-            if (round == 0) hist_add(hist, key >> 21, in);
-            else hist_add(hist, (key >> 10) & 0x7FFu, in && (key >> 21) == b1);
-        }
-    }
-}
-
-__global__ void __launch_bounds__(32 * kThrWarps)
+// One warp per row: tau[r] = the rank-th largest sampled order key, rank = e + 6 sqrt(e) + 2
+// for the e = k * m / n samples expected above the row's k-th largest score.  The row's
+// at most 2048 samples sit in registers (64 per lane) and the key is found bit by bit from
+// the top: 32 counting passes of ballot-free compares and a warp sum, no shared memory.
+// The first CTA also clears the window's fallback flag.
+__global__ void __launch_bounds__(32 * kRowWarps)
 topk_threshold_kernel(const float* __restrict__ sample, long long ld_sample, int q_begin,
                       int rows, int tile_stride, int k, uint32_t* __restrict__ tau,
                       int* __restrict__ fb_any) {
-    __shared__ uint32_t hist_all[kThrWarps][kThrBins];
+    constexpr int kPer = kSampleMax / 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (blockIdx.x == 0 && threadIdx.x == 0) *fb_any = 0;
-    const int r = blockIdx.x * kThrWarps + warp;
+    const int r = blockIdx.x * kRowWarps + warp;
     if (r >= rows) return;
-    uint32_t* hist = hist_all[warp];
     const int t = q_begin + r;
     const int n = t + 1;
     // valid samples: logical tile j holds keys j*stride*128 .. +127, causal ones only
@@ -571,21 +521,22 @@ topk_threshold_kernel(const float* __restrict__ sample, long long ld_sample, int
     uint32_t rank = (uint32_t)ceilf(e + 6.f * sqrtf(e)) + 2u;
     if (rank > (uint32_t)m) rank = (uint32_t)m;
     const float* row = sample + (long long)r * ld_sample;
-    for (int i = lane; i < kThrBins; i += 32) hist[i] = 0u;
-    __syncwarp();
-    threshold_pass(row, ncols, span, t, hist, 0, 0u);  // bits 31..21
-    __syncwarp();
-    uint32_t b1, above;
-    warp_find_bin(hist, rank, &b1, &above);
-    const uint32_t need2 = rank - above;
-    __syncwarp();
-    for (int i = lane; i < kThrBins; i += 32) hist[i] = 0u;
-    __syncwarp();
-    threshold_pass(row, ncols, span, t, hist, 1, b1);  // bits 20..10 within bin b1
-    __syncwarp();
-    uint32_t b2, above2;
-    warp_find_bin(hist, need2, &b2, &above2);
-    if (lane == 0) tau[r] = (b1 << 21) | (b2 << 10);
+    uint32_t key[kPer];  // 0 marks a missing sample (below every real order key)
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int c = i * 32 + lane;
+        const bool in = c < ncols && (c / kBM_SAMPLE) * span + (c % kBM_SAMPLE) <= t;
+        key[i] = in ? float_order_key(__ldg(row + c)) : 0u;
+    }
+    uint32_t prefix = 0u;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = prefix | (1u << bit);
+        uint32_t cnt = 0;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) cnt += key[i] >= cand ? 1u : 0u;
+        if (warp_sum(cnt) >= rank) prefix = cand;
+    }
+    if (lane == 0) tau[r] = prefix;
 }
 
 // One CTA per row: the exact top-k among the row's candidates (all keys at or above
@@ -683,11 +634,13 @@ cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin
     return cudaGetLastError();
 }
 
+int topk_sample_max() { return kSampleMax; }
+
 cudaError_t launch_topk_threshold(const float* sample, long long ld_sample, int q_begin, int rows,
                                   int tile_stride, int k, uint32_t* tau, int* fb_any,
                                   cudaStream_t stream) {
-    const int grid = (rows + kThrWarps - 1) / kThrWarps;
-    topk_threshold_kernel<<<grid, 32 * kThrWarps, 0, stream>>>(sample, ld_sample, q_begin, rows,
+    const int grid = (rows + kRowWarps - 1) / kRowWarps;
+    topk_threshold_kernel<<<grid, 32 * kRowWarps, 0, stream>>>(sample, ld_sample, q_begin, rows,
                                                                 tile_stride, k, tau, fb_any);
     count_launch(DSA_KERNEL_TOPK);
     return cudaGetLastError();
