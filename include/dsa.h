@@ -54,7 +54,7 @@ typedef struct CUstream_st* dsa_stream_t; /* same type as cudaStream_t */
 typedef enum {
     DSA_OK = 0,
     DSA_ERR_INVALID_ARG = 1,  /* a pointer, size, stride or alignment is wrong */
-    DSA_ERR_UNSUPPORTED = 2,  /* a valid request this build has no kernel for */
+    DSA_ERR_UNSUPPORTED = 2,  /* a valid request the library has no kernel for */
     DSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
     DSA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
     DSA_ERR_DEVICE_CHECK = 5  /* a kernel recorded an invalid input (see error bits) */
