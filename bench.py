@@ -531,7 +531,8 @@ def run_reference(args, rank, world):
     value = rows / secs
     return {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 0,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / value, 3),
+        # a step is the whole T-token prefill, at the sampled rate
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(T * 1e3 / value, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
         "config": {"workload": f"dsa_prefill_T{T}_top{k}", "T": T, "topk": k},
