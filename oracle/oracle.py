@@ -244,3 +244,86 @@ def pattern_from_freq(freq: int, num_layers: int) -> str:
     if freq < 1 or num_layers < 1:
         raise ValueError("freq and num_layers must be positive")
     return "".join("F" if i % freq == 0 else "S" for i in range(num_layers))
+
+
+# ---------------------------------------------------------------------------------
+# fp8 latent cache
+# ---------------------------------------------------------------------------------
+# DeepSeek-V2-Lite-Chat SIQ card (what is quantized, KV-cache bullet): the non-sparse MLA
+# backend keeps the KV cache in fp8 at 576 bytes per token, i.e. one byte for each of the
+# 576 latent elements.  The card does not spell out the encoding; the reading here is the
+# E4M3 variant of the OCP 8-bit floating-point format with one fp32 scale per cache
+# tensor, value = kv_scale * e4m3(code).
+#
+# E4M3 (OCP 8-bit floating point specification): bit 7 sign, bits 6..3 exponent with
+# bias 7, bits 2..0 mantissa.  Exponent field 0 encodes subnormals m/8 * 2^-6; the code
+# with exponent and mantissa fields all ones (0x7f / 0xff) is NaN; there is no infinity,
+# so the largest finite magnitude is 1.75 * 2^8 = 448.
+#
+# Mutants 9..12 (Python-side planted mistakes for the pin mutation test):
+#   9  exponent bias 8 instead of 7        10  subnormals decoded as normals
+#   11 encoder ties rounded away from zero 12  kv_scale left off the attention output
+def e4m3_decode(codes, mutant: int = 0) -> np.ndarray:
+    """Exact float64 values of E4M3 codes (uint8 array of any shape)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = (c >> 7) & 1
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    bias = 8 if mutant == 9 else 7
+    normal = (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - bias)
+    sub = (m / 8.0) * 2.0 ** (1 - bias)
+    mag = normal if mutant == 10 else np.where(e == 0, sub, normal)
+    val = np.where(sign == 1, -mag, mag)
+    return np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def e4m3_encode(x, mutant: int = 0) -> np.ndarray:
+    """E4M3 codes of float values, rounded to the nearest code with ties to the even code
+    (round-to-nearest-even), magnitudes above 448 saturated to 448 (the finite-saturating
+    conversion), the sign kept for values that round to zero; NaN -> 0x7f."""
+    xs = np.asarray(x, dtype=np.float64)
+    pos = e4m3_decode(np.arange(127, dtype=np.uint8), mutant)  # codes 0..126: 0 .. 448
+    a = np.abs(xs)
+    hi_i = np.clip(np.searchsorted(pos, a, side="left"), 1, 126)
+    lo_i = hi_i - 1
+    lo, hi = pos[lo_i], pos[hi_i]
+    mid = (lo + hi) / 2.0  # exact: both are short binary fractions
+    if mutant == 11:
+        tie = hi_i
+    else:
+        tie = np.where(lo_i % 2 == 0, lo_i, hi_i)
+    code = np.where(a < mid, lo_i, np.where(a > mid, hi_i, tie))
+    code = np.where(a >= pos[126], 126, code)
+    code = code | (np.signbit(xs).astype(np.int64) << 7)
+    code = np.where(np.isnan(xs), 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def latent_quantize_fp8(c, kv_scale: float, mutant: int = 0) -> np.ndarray:
+    """Codes of a latent cache: e4m3_encode(c / kv_scale), the quotient taken in fp32
+    (the precision in which the quantised code is decided)."""
+    x = _f32(c) / np.float32(kv_scale)
+    return e4m3_encode(x.astype(np.float32), mutant)
+
+
+def sparse_mla_fp8_prefill(q, kv_codes, kv_scale: float, idx, scale: float, d_v: int = 512,
+                           mutant: int = 0):
+    """Absorbed MLA over an fp8 latent cache: the latent row of key s is
+    kv_scale * e4m3_decode(kv_codes[s]).  The decoded codes are exact in float32, so the
+    attention runs on them with the logit scale scale*kv_scale, and the output (a convex
+    combination of value rows) is multiplied by kv_scale."""
+    codes = kv_codes.detach().cpu().numpy() if hasattr(kv_codes, "detach") else kv_codes
+    c = e4m3_decode(codes, mutant).astype(np.float32)
+    out, lse = sparse_mla_prefill(q, c, idx, float(scale) * float(kv_scale), d_v, mutant)
+    return (out if mutant == 12 else out * float(kv_scale)), lse
+
+
+def sparse_mla_fp8_decode(q, kv_pool_codes, kv_scale: float, page_table, idx, scale: float,
+                          d_v: int = 512, mutant: int = 0):
+    """Decode over a paged fp8 latent pool [num_pages, page_size, D_qk] of E4M3 codes."""
+    codes = (kv_pool_codes.detach().cpu().numpy() if hasattr(kv_pool_codes, "detach")
+             else kv_pool_codes)
+    c = e4m3_decode(codes, mutant).astype(np.float32)
+    out, lse = sparse_mla_decode(q, c, page_table, idx, float(scale) * float(kv_scale), d_v,
+                                 mutant)
+    return (out if mutant == 12 else out * float(kv_scale)), lse

@@ -16,6 +16,10 @@ context 3072; MLA latent 576 = 512 + 64 from the DeepSeek-V2-Lite-Chat SIQ card)
 * ``mla_prefill_gauss`` bf16, indexer q_idx/k_idx ~ N(0,1), w ~ U(0,1); q, kv as above.
 * ``mla_decode``     bf16, B sequences of length L over 64-token pages with a random
                      page permutation; integer indexer inputs as above.
+* ``*_fp8`` variants the latent cache as E4M3 codes (one byte per element, 576 bytes per
+                     token, DeepSeek-V2-Lite-Chat SIQ card) with one fp32 scale per cache:
+                     draws of N(0, (0.5/kv_scale)^2), clamped to +-448 and cast to
+                     torch.float8_e4m3fn, so that kv_scale * code ~ N(0, 0.5^2) as for bf16.
 """
 from __future__ import annotations
 
@@ -87,6 +91,31 @@ def mla_layer(T: int, seed: int, H: int = H_MLA, D: int = D_QK_MLA, g=None) -> d
             "kv": _normal(g, 0.5, (T, D), torch.bfloat16)}
 
 
+KV_SCALE_FP8 = 2.0 ** -7
+
+
+def _e4m3_codes(g, std: float, shape, chunk: int = 1 << 26) -> torch.Tensor:
+    """uint8 E4M3 codes of N(0, std^2) draws clamped to +-448 (a dtype cast per chunk)."""
+    n = 1
+    for s in shape:
+        n *= s
+    out = torch.empty(n, dtype=torch.uint8)
+    for i in range(0, n, chunk):
+        m = min(chunk, n - i)
+        z = (torch.randn(m, generator=g, dtype=torch.float32) * std).clamp_(-448.0, 448.0)
+        out[i:i + m] = z.to(torch.float8_e4m3fn).view(torch.uint8)
+    return out.view(*shape)
+
+
+def mla_layer_fp8(T: int, seed: int, kv_scale: float = KV_SCALE_FP8, H: int = H_MLA,
+                  D: int = D_QK_MLA, g=None) -> dict:
+    """MLA inputs over an fp8 latent cache: q [T,H,D] bf16 ~ N(0, 0.5^2); kv [T,D] uint8
+    E4M3 codes with kv_scale * value ~ N(0, 0.5^2)."""
+    g = g or _gen(seed)
+    return {"q": _normal(g, 0.5, (T, H, D), torch.bfloat16),
+            "kv": _e4m3_codes(g, 0.5 / kv_scale, (T, D)), "kv_scale": kv_scale}
+
+
 def mla_prefill_int(T: int = 8192, seed: int = 0, k: int = 2048) -> dict:
     g = _gen(seed)
     d = indexer_int(T, seed, g=g)
@@ -99,6 +128,16 @@ def mla_prefill_gauss(T: int = 65536, seed: int = 0, k: int = 2048) -> dict:
     g = _gen(seed)
     d = indexer_gauss(T, seed, g=g)
     d.update(mla_layer(T, seed, g=g))
+    d.update(T=T, topk=k, scale=SCALE_MLA)
+    return d
+
+
+def mla_prefill_gauss_fp8(T: int = 65536, seed: int = 0, k: int = 2048,
+                          kv_scale: float = KV_SCALE_FP8) -> dict:
+    """mla_prefill_gauss with the latent cache as E4M3 codes."""
+    g = _gen(seed)
+    d = indexer_gauss(T, seed, g=g)
+    d.update(mla_layer_fp8(T, seed, kv_scale, g=g))
     d.update(T=T, topk=k, scale=SCALE_MLA)
     return d
 
@@ -139,4 +178,24 @@ def mla_decode(B: int = 64, L: int = 32768, seed: int = 0, k: int = 2048,
         seq_lens = [L] * B
     d["seq_lens"] = torch.tensor(seq_lens, dtype=torch.int32)
     d.update(B=B, L=L, topk=k, page_size=page_size, scale=SCALE_MLA)
+    return d
+
+
+def mla_decode_fp8(B: int = 64, L: int = 32768, seed: int = 0, k: int = 2048,
+                   page_size: int = 64, seq_lens=None, kv_scale: float = KV_SCALE_FP8) -> dict:
+    """mla_decode with the paged latent pool as E4M3 codes (same order of draws)."""
+    g = _gen(seed)
+    max_pages = (L + page_size - 1) // page_size
+    num_pages = B * max_pages
+    d = {}
+    d["q_idx"] = _randint(g, -4, 4, (B, H_I_MLA, D_I_MLA), torch.bfloat16)
+    d["w"] = _randint(g, 1, 3, (B, H_I_MLA), torch.float32)
+    d["k_idx_pool"] = _randint(g, -4, 4, (num_pages, page_size, D_I_MLA), torch.bfloat16)
+    d["q"] = _normal(g, 0.5, (B, H_MLA, D_QK_MLA), torch.bfloat16)
+    d["kv_pool"] = _e4m3_codes(g, 0.5 / kv_scale, (num_pages, page_size, D_QK_MLA))
+    d["page_table"] = torch.randperm(num_pages, generator=g).to(torch.int32).view(B, max_pages)
+    if seq_lens is None:
+        seq_lens = [L] * B
+    d["seq_lens"] = torch.tensor(seq_lens, dtype=torch.int32)
+    d.update(B=B, L=L, topk=k, page_size=page_size, scale=SCALE_MLA, kv_scale=kv_scale)
     return d

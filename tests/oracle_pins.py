@@ -321,4 +321,119 @@ def pin_causal_prefix_invariance(mutant=0):
     assert O.prefill_indices(q1, k1, w1, 1, mutant=mutant)[2, 0] == 2
 
 
+
+# ---------------------------------------------------------------------------------
+# fp8 (E4M3) latent cache
+# ---------------------------------------------------------------------------------
+def _torch_e4m3_values(codes):
+    """Library decode of E4M3 codes (torch.float8_e4m3fn) as float64."""
+    t = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def pin_e4m3_decode(mutant=0):
+    """Every one of the 256 codes decodes to torch.float8_e4m3fn's value (NaN codes
+    0x7f/0xff included), and a few codes to the closed forms of the format: 0x01 is the
+    smallest subnormal 2^-9, 0x08 the smallest normal 2^-6, 0x38 is 1, 0x7e is 448."""
+    codes = np.arange(256, dtype=np.uint8)
+    v = O.e4m3_decode(codes, mutant)
+    t = _torch_e4m3_values(codes)
+    assert np.array_equal(np.isnan(v), np.isnan(t))
+    fin = ~np.isnan(t)
+    assert np.array_equal(v[fin], t[fin])
+    assert np.array_equal(np.signbit(v[fin]), np.signbit(t[fin]))
+    forms = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0,
+             0x3C: 1.5, 0x7E: 448.0, 0xFE: -448.0, 0xB8: -1.0}
+    for c, val in forms.items():
+        assert O.e4m3_decode(np.array([c], np.uint8), mutant)[0] == val, hex(c)
+    assert np.isnan(O.e4m3_decode(np.array([0x7F], np.uint8), mutant)[0])
+
+
+def pin_e4m3_encode(mutant=0):
+    """Encoding agrees with torch's float32 -> float8_e4m3fn conversion (round to nearest
+    even) wherever that conversion is finite (|x| < 448 here), including values exactly
+    halfway between neighbouring codes and subnormal magnitudes; brute force (the nearest
+    of all finite codes, ties to the even code) agrees too; magnitudes above 448
+    saturate to 448 (0x7e / 0xfe); decode(encode(v)) = v for every finite code."""
+    r = _rng(30)
+    pos = _torch_e4m3_values(np.arange(127, dtype=np.uint8))
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)
+    x = np.concatenate([
+        (r.normal(size=4000) * 60).astype(np.float32),
+        (r.normal(size=2000) * 2.0 ** -8).astype(np.float32),
+        mids, -mids, pos.astype(np.float32), np.float32([0.0, -0.0, 447.9, -447.9])])
+    x = x[np.abs(x) < 448]
+    c = O.e4m3_encode(x, mutant)
+    t = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(c, t), np.nonzero(c != t)
+    allv = _torch_e4m3_values(np.arange(256, dtype=np.uint8))
+    fin_codes = np.nonzero(~np.isnan(allv))[0]
+    xs = x[:600].astype(np.float64)
+    d = np.abs(xs[:, None] - allv[fin_codes][None, :])
+    best = d.min(axis=1, keepdims=True)
+    for i in range(len(xs)):
+        cand = fin_codes[d[i] == best[i, 0]]
+        cand = cand[np.signbit(allv[cand]) == np.signbit(xs[i])] if len(cand) > 1 else cand
+        want = cand[(cand & 1) == 0][0] if len(cand) > 1 else cand[0]
+        assert c[i] == want, (xs[i], c[i], want)
+    sat = O.e4m3_encode(np.float32([449.0, 500.0, 1e6, -464.0, -3e38]), mutant)
+    assert sat.tolist() == [0x7E, 0x7E, 0x7E, 0xFE, 0xFE]
+    fin = np.nonzero(~np.isnan(allv))[0].astype(np.uint8)
+    assert np.array_equal(O.e4m3_encode(allv[fin].astype(np.float32), mutant), fin)
+
+
+def pin_latent_quantize(mutant=0):
+    """Quantising a bf16 latent row: the fp32 quotient c / kv_scale, then the library's
+    round-to-nearest-even E4M3 conversion (values kept inside +-448)."""
+    r = _rng(31)
+    c = torch.from_numpy((0.5 * r.normal(size=(64, 576))).astype(np.float32)).to(torch.bfloat16)
+    for s in (2.0 ** -7, 0.0123):
+        got = O.latent_quantize_fp8(c, s, mutant)
+        ref = (c.float() / torch.tensor(s, dtype=torch.float32)).clamp(-448, 448)
+        ref = ref.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(got, ref)
+
+
+def pin_fp8_attention_masked_sdpa(mutant=0):
+    """Attention over an fp8 latent cache equals torch SDPA (fp64) on the latent rows
+    decoded by the library (torch.float8_e4m3fn) and multiplied by kv_scale, under the
+    mask built from the indices; the log-sum-exp equals torch.logsumexp of the logits;
+    paged decode of the last query equals its prefill row."""
+    r = _rng(32)
+    T, H, D, k = 70, 2, 576, 24
+    q = (0.5 * r.normal(size=(T, H, D))).astype(np.float32)
+    codes = torch.from_numpy((64 * r.normal(size=(T, D))).clip(-440, 440).astype(np.float32))
+    codes = codes.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    idx = np.full((T, k), -1, dtype=np.int32)
+    mask = np.zeros((T, T), dtype=bool)
+    for t in range(T):
+        sel = np.sort(r.choice(t + 1, size=min(k, t + 1), replace=False))
+        idx[t, :len(sel)] = sel
+        mask[t, sel] = True
+    for s in (2.0 ** -7, 0.0123):
+        out, lse = O.sparse_mla_fp8_prefill(q, codes, s, idx, 192 ** -0.5, mutant=mutant)
+        c = _torch_e4m3_values(codes) * s
+        kk = np.repeat(c[:, None, :], H, axis=1)
+        ref = _sdpa64(q, kk, kk[..., :512], mask=mask, scale=192 ** -0.5)
+        np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+        logits = np.einsum("thd,sd->ths", q.astype(np.float64), c) * 192 ** -0.5
+        logits = np.where(mask[:, None, :], logits, -np.inf)
+        ref_lse = torch.logsumexp(torch.from_numpy(logits), dim=-1).numpy()
+        np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+    # paged decode: the pool is a permutation of 64-row pages of the same codes
+    ps, npg = 8, (T + 7) // 8
+    pool = np.zeros((npg * ps, D), np.uint8)
+    pool[:T] = codes
+    pool = pool.reshape(npg, ps, D)
+    perm = r.permutation(npg)
+    ppool = np.empty_like(pool)
+    ppool[perm] = pool
+    pt = perm.astype(np.int32)[None, :]
+    od, ld = O.sparse_mla_fp8_decode(q[T - 1:], ppool, 0.0123, pt, idx[T - 1:], 192 ** -0.5,
+                                     mutant=mutant)
+    op, lp = O.sparse_mla_fp8_prefill(q[T - 1:], codes, 0.0123, idx[T - 1:], 192 ** -0.5,
+                                      mutant=mutant)
+    np.testing.assert_allclose(od, op, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(ld, lp, rtol=1e-12, atol=1e-15)
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

@@ -32,3 +32,16 @@ def test_stack_seeds_per_layer():
     s = G.layer_stack(T=32, pattern="FSS")
     assert "q_idx" in s["layers"][0] and "q_idx" not in s["layers"][1]
     assert not torch.equal(s["layers"][0]["q"], s["layers"][1]["q"])
+
+
+def test_fp8_latent_codes():
+    """E4M3 codes: no NaN code, deterministic, and kv_scale * value ~ N(0, 0.5^2)."""
+    a, b = G.mla_layer_fp8(T=256, seed=3), G.mla_layer_fp8(T=256, seed=3)
+    assert a["kv"].dtype == torch.uint8 and a["kv"].shape == (256, 576)
+    assert torch.equal(a["kv"], b["kv"]) and torch.equal(a["q"], b["q"])
+    assert not bool(((a["kv"] & 0x7F) == 0x7F).any())
+    val = a["kv"].view(torch.float8_e4m3fn).to(torch.float32) * a["kv_scale"]
+    assert 0.45 < val.std().item() < 0.55
+    d = G.mla_decode_fp8(B=2, L=130, page_size=64)
+    assert d["kv_pool"].shape == (6, 64, 576) and d["kv_pool"].dtype == torch.uint8
+    assert torch.equal(d["page_table"], G.mla_decode(B=2, L=130, page_size=64)["page_table"])

@@ -1,6 +1,7 @@
 """Mutation check of the pins: each deliberate mistake compiled into the oracle
 (ORACLE_MUTANT in dsa_oracle.c) must make at least one pin fail.  The mistakes are
-planted only in CPU builds of the oracle."""
+planted only in CPU builds of the oracle (mutants 9..12 in the oracle's Python fp8
+functions)."""
 import pytest
 
 import oracle_pins as P
@@ -15,6 +16,10 @@ MUTANTS = {
     6: "softmax scale dropped",
     7: "value read from the wrong slice",
     8: "lse without the max",
+    9: "E4M3 exponent bias 8",
+    10: "E4M3 subnormals decoded as normals",
+    11: "E4M3 encoder ties away from zero",
+    12: "fp8 attention output without kv_scale",
 }
 
 
