@@ -20,6 +20,7 @@ import sys
 import time
 from pathlib import Path
 
+
 ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
@@ -41,6 +42,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", choices=["prefill", "decode", "stack"], default="prefill",
                     help="prefill: the T=65536 headline; decode: 64 sequences x 32768 paged "
                          "tokens; stack: the 27-layer FSS x 9 IndexCache stack at T=16384")
+    ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
+                    help="latent cache: bf16, or E4M3 codes times one fp32 scale")
     ap.add_argument("--window-rows", type=int, default=0,
                     help="query rows per indexer/top-k window (0 = the library default)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -51,22 +54,25 @@ def parse_args(argv=None):
 # ----------------------------------------------------------------------------------
 # workload
 # ----------------------------------------------------------------------------------
-def make_inputs(T, k, seed):
+def make_inputs(T, k, seed, kv_dtype="bf16"):
     from sparse_attention_17_b200 import inputs as G
+    if kv_dtype == "fp8":
+        return G.mla_prefill_gauss_fp8(T=T, seed=seed, k=k)
     return G.mla_prefill_gauss(T=T, seed=seed, k=k)
 
 
-def algorithmic_work(T, k):
-    """FLOPs and bytes of one prefill step, counted from the definitions."""
+def algorithmic_work(T, k, kv_bytes=2):
+    """FLOPs and bytes of one prefill step, counted from the definitions (kv_bytes: bytes
+    per latent element, 2 for bf16, 1 for E4M3 codes)."""
     causal = T * (T + 1) // 2                       # (t, s) pairs with s <= t
     sel = sum(min(t + 1, k) for t in range(T))      # selected keys over all queries
     return {
         "indexer_flop": 2 * 16 * 64 * causal,       # 16 heads x 64-dim dot per pair
         "mla_flop": 2 * 16 * (576 + 512) * sel,     # QK (576) + PV (512) per head per key
-        "mla_gather_bytes": 1152 * sel,             # one 576 x bf16 latent row per key
+        "mla_gather_bytes": 576 * kv_bytes * sel,   # one 576-element latent row per key
         "topk_read_bytes": 4 * causal,              # fp32 scores read once per pair
         "hbm_bytes": (T * 16 * 64 * 2 + T * 64 * 2 + T * 16 * 4 + T * 16 * 576 * 2
-                      + T * 576 * 2 + T * 16 * 512 * 2 + 2 * T * k * 4),
+                      + T * 576 * kv_bytes + T * 16 * 512 * 2 + 2 * T * k * 4),
     }
 
 
@@ -190,7 +196,9 @@ def oracle_rows_throughput(d, k, seconds, rng_seed=0, max_rows=None):
     T = d["q_idx"].shape[0]
     r = np.random.default_rng(rng_seed)
     q_idx, k_idx, w = (O._f32(d[n]) for n in ("q_idx", "k_idx", "w"))
-    q, kv = d["q"], O._f32(d["kv"])
+    fp8 = "kv_scale" in d
+    q = d["q"]
+    kv = d["kv"].numpy() if fp8 else O._f32(d["kv"])
     threads = O.num_threads()
     block = 2 * threads
     done, t0 = 0, time.perf_counter()
@@ -198,7 +206,10 @@ def oracle_rows_throughput(d, k, seconds, rng_seed=0, max_rows=None):
         b0 = int(r.integers(0, T - block + 1))
         sc = O.indexer_scores_prefill(q_idx, k_idx, w, b0, block, b0 + block)
         idx = O.topk(sc, O.causal_n_valid(b0, block), k)
-        O.sparse_mla_prefill(q[b0:b0 + block], kv, idx, 192 ** -0.5)
+        if fp8:
+            O.sparse_mla_fp8_prefill(q[b0:b0 + block], kv, d["kv_scale"], idx, 192 ** -0.5)
+        else:
+            O.sparse_mla_prefill(q[b0:b0 + block], kv, idx, 192 ** -0.5)
         done += block
         el = time.perf_counter() - t0
         if el >= seconds or (max_rows and done >= max_rows):
@@ -220,7 +231,8 @@ def run_native(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     plan = shard_plan(rank, world, args.T, args.topk)
     T, k = plan["T"], plan["topk"]
-    host = make_inputs(T, k, seed=plan["seed"])
+    fp8 = args.kv_dtype == "fp8"
+    host = make_inputs(T, k, seed=plan["seed"], kv_dtype=args.kv_dtype)
     names = ("q_idx", "k_idx", "w", "q", "kv")
     x = {n: host[n].to(dev) for n in names}
     ld = (T + 3) // 4 * 4
@@ -243,7 +255,10 @@ def run_native(args, rank, world, local_rank):
             dsa.topk_select(scores, k, idx[q0:q0 + rows], q_begin=q0, rows=rows)
         if ev is not None:
             ev[1].record(stream)
-        dsa.sparse_mla_fwd(xin["q"], xin["kv"], idx, o, G.SCALE_MLA)
+        if fp8:
+            dsa.sparse_mla_fp8_fwd(xin["q"], xin["kv"], host["kv_scale"], idx, o, G.SCALE_MLA)
+        else:
+            dsa.sparse_mla_fwd(xin["q"], xin["kv"], idx, o, G.SCALE_MLA)
         if ev is not None:
             ev[2].record(stream)
 
@@ -263,7 +278,7 @@ def run_native(args, rank, world, local_rank):
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches0 = [dsa.launch_count(i) for i in range(4)]
+    launches0 = [dsa.launch_count(i) for i in range(dsa.KERNEL_KINDS)]
     with ClockSampler(local_rank) as clk:
         sync_all()
         start.record(stream)
@@ -271,7 +286,7 @@ def run_native(args, rank, world, local_rank):
             step(evs[i])
         stop.record(stream)
         torch.cuda.synchronize()
-    launches = sum(dsa.launch_count(i) - launches0[i] for i in range(4))
+    launches = sum(dsa.launch_count(i) - launches0[i] for i in range(dsa.KERNEL_KINDS))
     ms_total = start.elapsed_time(stop)
     idx_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     mla_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
@@ -349,7 +364,7 @@ def run_native(args, rank, world, local_rank):
 
     result = None
     if rank == 0:
-        work = algorithmic_work(T, k)
+        work = algorithmic_work(T, k, kv_bytes=1 if fp8 else 2)
         peaks, peak_src = load_peaks()
         ms_step = ms_total / args.steps
         value = aggregate_tokens_per_s(T, world, ms_step)
@@ -366,7 +381,7 @@ def run_native(args, rank, world, local_rank):
         achieved = flop / (dom_ms / 1e3) / 1e12
         roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 2),
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                    "traffic": load_traffic(fname),
+                    "traffic": load_traffic(fname + (":fp8" if fp8 else "")),
                     "peak_source": f"{peak_src} bf16 dense, sustained (kernel timed inside a long step)"}
         others = {
             "indexer_tflops": round(work["indexer_flop"] / (indexer_ms / 1e3) / 1e12, 2),
@@ -382,9 +397,11 @@ def run_native(args, rank, world, local_rank):
         result = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8-e4m3 latent cache, f16 MMAs" if fp8 else "bf16",
             "data": "synthetic",
-            "config": {"workload": f"dsa_prefill_T{T}_top{k}", "T": T, "topk": k,
+            "config": {"workload": f"dsa_prefill_T{T}_top{k}" + ("_fp8kv" if fp8 else ""),
+                       "T": T, "topk": k, "kv_cache": "e4m3 x kv_scale" if fp8 else "bf16",
                        "batch_per_gpu": 1, "indexer_heads": 16, "indexer_dim": 64,
                        "heads": 16, "latent_dim": 576, "value_dim": 512,
                        "index_window_rows": rw, "parallelism": f"independent sequences x{world}",
@@ -435,7 +452,8 @@ def run_decode(args, local_rank):
     from sparse_attention_17_b200 import inputs as G
     torch.cuda.set_device(local_rank)
     B, L, k = 64, 32768, args.topk
-    host = G.mla_decode(B=B, L=L, k=k)
+    fp8 = args.kv_dtype == "fp8"
+    host = G.mla_decode_fp8(B=B, L=L, k=k) if fp8 else G.mla_decode(B=B, L=L, k=k)
     x = {n: host[n].cuda() for n in ("q_idx", "w", "k_idx_pool", "q", "kv_pool", "page_table",
                                       "seq_lens")}
     scores = torch.empty((B, L), dtype=torch.float32, device="cuda")
@@ -452,8 +470,13 @@ def run_decode(args, local_rank):
         dsa.topk_select(scores, k, idx, row_len=x["seq_lens"], max_len=L)
 
     def mla():
-        dsa.sparse_mla_fwd(x["q"], x["kv_pool"], idx, out, G.SCALE_MLA, page_table=x["page_table"],
-                           seq_lens=x["seq_lens"], workspace=ws)
+        if fp8:
+            dsa.sparse_mla_fp8_fwd(x["q"], x["kv_pool"], host["kv_scale"], idx, out, G.SCALE_MLA,
+                                   page_table=x["page_table"], seq_lens=x["seq_lens"],
+                                   workspace=ws)
+        else:
+            dsa.sparse_mla_fwd(x["q"], x["kv_pool"], idx, out, G.SCALE_MLA,
+                               page_table=x["page_table"], seq_lens=x["seq_lens"], workspace=ws)
 
     def step():
         indexer(); topk(); mla()
@@ -464,13 +487,14 @@ def run_decode(args, local_rank):
     t_mla = _timed(mla, args.steps, 1, stream)
     assert dsa.check_device_errors() == 0
     peaks, src = load_peaks()
-    gather = B * k * 1152
+    gather = B * k * (576 if fp8 else 1152)
     kidx = B * L * 64 * 2
     return {"metric": "DSA decode sequences/sec (64 x 32768 paged, top-2048)", "value":
             round(B / (ms / 1e3), 1), "unit": "sequences/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-            "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "dsa_decode_B64_L32768_top2048", "page_size": 64},
+            "dtype": "fp8-e4m3 latent cache, f16 MMAs" if fp8 else "bf16", "data": "synthetic",
+            "config": {"workload": "dsa_decode_B64_L32768_top2048" + ("_fp8kv" if fp8 else ""),
+                       "page_size": 64, "kv_cache": "e4m3 x kv_scale" if fp8 else "bf16"},
             "kernels": {"indexer_ms": round(t_idx, 4), "topk_ms": round(t_topk, 4),
                         "sparse_mla_decode_ms": round(t_mla, 4)},
             "derived": {"indexer_key_read_gbs": round(kidx / (t_idx / 1e3) / 1e9, 1),

@@ -11,6 +11,9 @@
  *                        512 dims; or plain multi-head attention for the fp32 path)
  *   dsa_layer_stack      an F/S pattern of layers: F layers run indexer + top-k into one
  *                        index buffer, S layers reuse it (IndexCache)
+ *   dsa_sparse_mla_fp8_fwd, dsa_latent_quantize_fp8
+ *                        the same attention over an fp8 (E4M3) latent cache, and the
+ *                        conversion of bf16 latent rows into such a cache
  *
  * Sources.  DSA ablation model card ("Attention" bullet: a ReLU lightning indexer picks the
  * top-k keys per query; closing note: prompts no longer than k attend densely);
@@ -60,7 +63,7 @@ typedef enum {
     DSA_ERR_DEVICE_CHECK = 5  /* a kernel recorded an invalid input (see error bits) */
 } dsa_status;
 
-typedef enum { DSA_F32 = 0, DSA_BF16 = 1 } dsa_dtype;
+typedef enum { DSA_F32 = 0, DSA_BF16 = 1, DSA_FP8_E4M3 = 2 } dsa_dtype;
 typedef enum { DSA_PREFILL = 0, DSA_DECODE = 1 } dsa_mode;
 
 /* Bits of the per-device error word (dsa_check_device_errors). */
@@ -74,7 +77,8 @@ typedef enum {
     DSA_KERNEL_TOPK = 1,
     DSA_KERNEL_ATTENTION = 2,
     DSA_KERNEL_COMBINE = 3,
-    DSA_KERNEL_KINDS = 4
+    DSA_KERNEL_QUANTIZE = 4,
+    DSA_KERNEL_KINDS = 5
 } dsa_kernel_kind;
 
 /* Human-readable name of a status code (static storage). */
@@ -226,6 +230,46 @@ dsa_status dsa_sparse_mla_decode_noalloc(int num_q, int H, int D_qk, int D_v, fl
                                          const int* seq_lens, const int* idx, int k_sel,
                                          long long ld_idx, void* out, float* lse,
                                          dsa_stream_t stream);
+
+/*
+ * dsa_sparse_mla_fp8_fwd -- dsa_sparse_mla_fwd (absorbed MLA, bf16 query, prefill or paged
+ * decode) over an fp8 latent cache.  DeepSeek-V2-Lite-Chat SIQ card (what is quantized,
+ * KV-cache bullet): fp8 KV at 576 bytes per token, one byte per latent element.
+ *
+ * Encoding (the card names only "fp8"; this is the reading used): each byte of `kv` is
+ * an E4M3 code of the OCP 8-bit floating-point format (sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, subnormals, 0x7f/0xff NaN, largest finite 448), and the latent element
+ * is kv_scale * E4M3(code), with one fp32 kv_scale for the whole cache.  So
+ *   logit_s = scale * kv_scale * q[n,h,:] . E4M3(kv[s,:])
+ *   out[n,h,:] = kv_scale * sum_s softmax_s(logit) * E4M3(kv[s, 0:512])
+ * kv [kv_rows, 576] uint8 (prefill) or [kv_rows / page_size, page_size, 576] (decode);
+ * every other argument, the supported shapes (H = 16, D_qk = 576, D_v = 512), the
+ * workspace (dsa_sparse_mla_workspace_size) and the error behaviour are those of
+ * dsa_sparse_mla_fwd with dtype DSA_BF16.
+ * Precision: the codes are widened exactly to f16 and the query is rounded to f16 for
+ * the tensor-core products (bf16 query values must lie within +-65504; magnitudes below
+ * 2^-14 keep f16's subnormal precision); probabilities are rounded to f16; fp32
+ * accumulation; out rounded to bf16.  kv_scale must be finite and > 0.  NaN codes are
+ * not supported.
+ */
+dsa_status dsa_sparse_mla_fp8_fwd(int mode, int num_q, int H, int D_qk, int D_v, float scale,
+                                  float kv_scale, const void* q, const void* kv,
+                                  long long kv_rows, const int* page_table, int max_pages,
+                                  int page_size, const int* seq_lens, const int* idx,
+                                  int k_sel, long long ld_idx, void* out, float* lse,
+                                  void* workspace, size_t workspace_bytes,
+                                  dsa_stream_t stream);
+
+/*
+ * dsa_latent_quantize_fp8 -- writes an fp8 latent cache for dsa_sparse_mla_fp8_fwd:
+ *   dst[i] = E4M3(src[i] / kv_scale),  i = 0 .. n-1
+ * src bf16 [n], dst uint8 [n] (both 16-byte aligned device pointers; n >= 0, any value).
+ * The quotient is the fp32 IEEE division (round to nearest); the conversion rounds to the
+ * nearest E4M3 value with ties to the even code, keeps the sign of values that round to
+ * zero, and saturates finite magnitudes above 448 to +-448.  kv_scale finite and > 0.
+ */
+dsa_status dsa_latent_quantize_fp8(const void* src, long long n, float kv_scale, void* dst,
+                                   dsa_stream_t stream);
 
 /*
  * dsa_layer_stack -- IndexCache over an F/S layer pattern (vLLM IndexCache docs, "How It

@@ -19,9 +19,10 @@ _lib = None
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, \
     DSA_ERR_DEVICE_CHECK = range(6)
-DSA_F32, DSA_BF16 = 0, 1
+DSA_F32, DSA_BF16, DSA_FP8_E4M3 = 0, 1, 2
 DSA_PREFILL, DSA_DECODE = 0, 1
-KERNEL_INDEXER, KERNEL_TOPK, KERNEL_ATTENTION, KERNEL_COMBINE = range(4)
+KERNEL_INDEXER, KERNEL_TOPK, KERNEL_ATTENTION, KERNEL_COMBINE, KERNEL_QUANTIZE = range(5)
+KERNEL_KINDS = 5
 DEVERR_INDEX_RANGE, DEVERR_PAGE_RANGE, DEVERR_TIMEOUT = 1, 2, 4
 
 # (name, restype, argtypes) of every exported symbol, in header order.
@@ -39,6 +40,9 @@ SYMBOLS = [
     ("dsa_sparse_mla_workspace_size", _SZ, [_I, _I, _I, _I, _I]),
     ("dsa_sparse_mla_decode_noalloc", _I, [_I, _I, _I, _I, _F, _P, _P, _LL, _P, _I, _I, _P, _P, _I,
                                            _LL, _P, _P, _P]),
+    ("dsa_sparse_mla_fp8_fwd", _I, [_I, _I, _I, _I, _I, _F, _F, _P, _P, _LL, _P, _I, _I, _P, _P,
+                                    _I, _LL, _P, _P, _P, _SZ, _P]),
+    ("dsa_latent_quantize_fp8", _I, [_P, _LL, _F, _P, _P]),
     ("dsa_layer_stack", _I, [ctypes.c_char_p, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P,
                              _P, _P, _P, _P, _P, _SZ, _P]),
     ("dsa_layer_stack_workspace_size", _SZ, [_I, _I]),
@@ -236,6 +240,53 @@ def sparse_mla_fwd(q, kv, idx, out, scale: float, lse=None, v=None, page_table=N
                                       page_table.data_ptr(), page_table.shape[1], page_size,
                                       seq_lens.data_ptr(), idx.data_ptr(), k_sel, idx.stride(0),
                                       out.data_ptr(), _ptr(lse), ws_ptr, ws_bytes, _stream()))
+
+
+def sparse_mla_fp8_fwd(q, kv, kv_scale: float, idx, out, scale: float, lse=None,
+                       page_table=None, seq_lens=None, workspace=None) -> None:
+    """dsa_sparse_mla_fp8_fwd.  q [N,16,576] bf16; kv uint8 E4M3 codes [S,576] (prefill)
+    or page pool [num_pages,page_size,576] (decode, with page_table/seq_lens); latent
+    value = kv_scale * code; out [N,16,512] bf16."""
+    lib = load()
+    _need(q, torch.bfloat16, 3, "q")
+    _need(idx, torch.int32, 2, "idx")
+    _need(out, torch.bfloat16, 3, "out")
+    if lse is not None:
+        _need(lse, torch.float32, 2, "lse")
+    num_q, H, D_qk = q.shape
+    D_v = out.shape[2]
+    k_sel = idx.shape[1]
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    if page_table is None:
+        _need(kv, torch.uint8, 2, "kv")
+        _check(lib.dsa_sparse_mla_fp8_fwd(DSA_PREFILL, num_q, H, D_qk, D_v, scale, kv_scale,
+                                          q.data_ptr(), kv.data_ptr(), kv.shape[0], None, 0, 0,
+                                          None, idx.data_ptr(), k_sel, idx.stride(0),
+                                          out.data_ptr(), _ptr(lse), ws_ptr, ws_bytes, _stream()))
+    else:
+        _need(kv, torch.uint8, 3, "kv")
+        _need(page_table, torch.int32, 2, "page_table")
+        _need(seq_lens, torch.int32, 1, "seq_lens")
+        page_size = kv.shape[1]
+        _check(lib.dsa_sparse_mla_fp8_fwd(DSA_DECODE, num_q, H, D_qk, D_v, scale, kv_scale,
+                                          q.data_ptr(), kv.data_ptr(), kv.shape[0] * page_size,
+                                          page_table.data_ptr(), page_table.shape[1], page_size,
+                                          seq_lens.data_ptr(), idx.data_ptr(), k_sel,
+                                          idx.stride(0), out.data_ptr(), _ptr(lse), ws_ptr,
+                                          ws_bytes, _stream()))
+
+
+def latent_quantize_fp8(src, kv_scale: float, dst) -> None:
+    """dsa_latent_quantize_fp8: dst (uint8, same shape) = E4M3(src (bf16) / kv_scale)."""
+    lib = load()
+    if src.dtype != torch.bfloat16 or dst.dtype != torch.uint8:
+        raise TypeError("src must be bfloat16 and dst uint8")
+    if not (src.is_contiguous() and dst.is_contiguous()) or src.numel() != dst.numel():
+        raise ValueError("src and dst must be contiguous with the same number of elements")
+    _check(lib.dsa_latent_quantize_fp8(src.data_ptr(), src.numel(), kv_scale, dst.data_ptr(),
+                                       _stream()))
 
 
 def layer_stack_workspace_size(T: int, rows_window: int = 0) -> int:

@@ -4,6 +4,7 @@
 // anything when they are wrong; then it calls the launchers of the kernel files.
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -240,6 +241,50 @@ size_t dsa_sparse_mla_workspace_size(int mode, int num_q, int H, int D_v, int k_
     return (size_t)num_q * splits * H * ((size_t)D_v + 1) * sizeof(float);
 }
 
+namespace {
+
+// The absorbed-MLA path behind dsa_sparse_mla_fwd (bf16 cache) and dsa_sparse_mla_fp8_fwd.
+dsa_status mla_absorbed(bool fp8, float kv_scale, int mode, int num_q, int H, int D_qk, int D_v,
+                        float scale, const void* q, const void* kv, long long kv_rows,
+                        const int* page_table, int max_pages, int page_size,
+                        const int* seq_lens, const int* idx, int k_sel, long long ld_idx,
+                        void* out, float* lse, void* workspace, size_t workspace_bytes,
+                        cudaStream_t cs, const DevCtx& ctx) {
+    if (H != 16 || D_qk != 576 || D_v != 512)
+        return fail(DSA_ERR_UNSUPPORTED,
+                    "MLA path is absorbed MLA: H=16, one shared 576-dim latent, D_v=512");
+    if (k_sel > 2048 || (k_sel & 3) || (ld_idx & 3))
+        return fail(DSA_ERR_UNSUPPORTED, "MLA path: k_sel <= 2048 and k_sel, ld_idx multiples of 4");
+    cudaError_t e;
+    if (mode == DSA_PREFILL) {
+        if (page_table || seq_lens) return fail(DSA_ERR_INVALID_ARG, "prefill takes no pages");
+        e = launch_sparse_mla_mma(static_cast<const __nv_bfloat16*>(q), kv, fp8, kv_scale, kv_rows,
+                                  nullptr, 0, 0, nullptr, idx, k_sel, ld_idx, num_q, scale, 1,
+                                  static_cast<__nv_bfloat16*>(out), lse, nullptr, nullptr, cs, ctx);
+        return e == cudaSuccess ? DSA_OK : cuda_fail(e, "attention launch");
+    }
+    if (!page_table || !seq_lens) return fail(DSA_ERR_INVALID_ARG, "decode needs page_table and seq_lens");
+    if (page_size <= 0 || max_pages <= 0 || kv_rows % page_size)
+        return fail(DSA_ERR_INVALID_ARG, "kv_rows must be num_pages * page_size");
+    const int splits = mla_decode_splits(num_q, k_sel, ctx.num_sms);
+    const size_t need = (size_t)num_q * splits * H * ((size_t)D_v + 1) * sizeof(float);
+    if (!workspace || workspace_bytes < need)
+        return fail(DSA_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need,
+                    workspace_bytes);
+    if (!aligned16(workspace)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    float* o_part = static_cast<float*>(workspace);
+    float* lse_part = o_part + (size_t)num_q * splits * H * D_v;
+    e = launch_sparse_mla_mma(static_cast<const __nv_bfloat16*>(q), kv, fp8, kv_scale, kv_rows,
+                              page_table, max_pages, page_size, seq_lens, idx, k_sel, ld_idx,
+                              num_q, scale, splits, nullptr, nullptr, o_part, lse_part, cs, ctx);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    e = launch_mla_combine(o_part, lse_part, num_q, splits, static_cast<__nv_bfloat16*>(out), lse,
+                           cs);
+    return e == cudaSuccess ? DSA_OK : cuda_fail(e, "combine launch");
+}
+
+}  // namespace
+
 dsa_status dsa_sparse_mla_fwd(int dtype, int mode, int num_q, int H, int num_kv_heads,
                               int D_qk, int D_v, float scale, const void* q, const void* kv,
                               const void* v, long long kv_rows, const int* page_table,
@@ -257,56 +302,76 @@ dsa_status dsa_sparse_mla_fwd(int dtype, int mode, int num_q, int H, int num_kv_
         return fail(DSA_ERR_INVALID_ARG, "bad sizes");
     if (!(scale > 0.f) || scale != scale) return fail(DSA_ERR_INVALID_ARG, "scale must be > 0");
     if (mode != DSA_PREFILL && mode != DSA_DECODE) return fail(DSA_ERR_INVALID_ARG, "bad mode");
+    if (dtype == DSA_FP8_E4M3)
+        return fail(DSA_ERR_INVALID_ARG, "an fp8 cache needs its scale: use dsa_sparse_mla_fp8_fwd");
+    if (dtype != DSA_BF16 && dtype != DSA_F32) return fail(DSA_ERR_INVALID_ARG, "bad dtype");
     if (num_q == 0) return DSA_OK;
     DevCtx ctx;
     dsa_status st = check_stream_device(&ctx);
     if (st != DSA_OK) return st;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e;
     if (dtype == DSA_F32) {
         if (mode != DSA_PREFILL) return fail(DSA_ERR_UNSUPPORTED, "fp32 attention is prefill only");
         if (!v || num_kv_heads != H || D_qk != D_v || D_qk > 64 || H > 16)
             return fail(DSA_ERR_UNSUPPORTED, "fp32 path: MHA with v, D <= 64, H <= 16");
         if (page_table || seq_lens) return fail(DSA_ERR_INVALID_ARG, "prefill takes no pages");
-        e = launch_sparse_mha_f32(static_cast<const float*>(q), static_cast<const float*>(kv),
+        cudaError_t e = launch_sparse_mha_f32(static_cast<const float*>(q), static_cast<const float*>(kv),
                                   static_cast<const float*>(v), num_q, H, D_qk, scale, kv_rows,
                                   idx, k_sel, ld_idx, static_cast<float*>(out), lse, cs, ctx);
         return e == cudaSuccess ? DSA_OK : cuda_fail(e, "attention launch");
     }
-    if (dtype != DSA_BF16) return fail(DSA_ERR_INVALID_ARG, "bad dtype");
-    if (H != 16 || num_kv_heads != 1 || D_qk != 576 || D_v != 512 || v != nullptr)
-        return fail(DSA_ERR_UNSUPPORTED,
-                    "bf16 path is absorbed MLA: H=16, one shared 576-dim latent, D_v=512, v=NULL");
-    if (k_sel > 2048 || (k_sel & 3) || (ld_idx & 3))
-        return fail(DSA_ERR_UNSUPPORTED,
-                    "bf16 MLA path: k_sel <= 2048 and k_sel, ld_idx multiples of 4");
-    if (mode == DSA_PREFILL) {
-        if (page_table || seq_lens) return fail(DSA_ERR_INVALID_ARG, "prefill takes no pages");
-        e = launch_sparse_mla_mma(static_cast<const __nv_bfloat16*>(q),
-                                   static_cast<const __nv_bfloat16*>(kv), kv_rows, nullptr, 0, 0,
-                                   nullptr, idx, k_sel, ld_idx, num_q, scale, 1,
-                                   static_cast<__nv_bfloat16*>(out), lse, nullptr, nullptr, cs, ctx);
-        return e == cudaSuccess ? DSA_OK : cuda_fail(e, "attention launch");
-    }
-    if (!page_table || !seq_lens) return fail(DSA_ERR_INVALID_ARG, "decode needs page_table and seq_lens");
-    if (page_size <= 0 || max_pages <= 0 || kv_rows % page_size)
-        return fail(DSA_ERR_INVALID_ARG, "kv_rows must be num_pages * page_size");
-    const int splits = mla_decode_splits(num_q, k_sel, ctx.num_sms);
-    const size_t need = (size_t)num_q * splits * H * ((size_t)D_v + 1) * sizeof(float);
-    if (!workspace || workspace_bytes < need)
-        return fail(DSA_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need,
-                    workspace_bytes);
-    if (!aligned16(workspace)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
-    float* o_part = static_cast<float*>(workspace);
-    float* lse_part = o_part + (size_t)num_q * splits * H * D_v;
-    e = launch_sparse_mla_mma(static_cast<const __nv_bfloat16*>(q),
-                               static_cast<const __nv_bfloat16*>(kv), kv_rows, page_table,
-                               max_pages, page_size, seq_lens, idx, k_sel, ld_idx, num_q, scale,
-                               splits, nullptr, nullptr, o_part, lse_part, cs, ctx);
-    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-    e = launch_mla_combine(o_part, lse_part, num_q, splits, static_cast<__nv_bfloat16*>(out), lse,
-                           cs);
-    return e == cudaSuccess ? DSA_OK : cuda_fail(e, "combine launch");
+    if (num_kv_heads != 1 || v != nullptr)
+        return fail(DSA_ERR_UNSUPPORTED, "bf16 path is absorbed MLA: one shared latent, v=NULL");
+    return mla_absorbed(false, 1.f, mode, num_q, H, D_qk, D_v, scale, q, kv, kv_rows, page_table,
+                        max_pages, page_size, seq_lens, idx, k_sel, ld_idx, out, lse, workspace,
+                        workspace_bytes, cs, ctx);
+}
+
+dsa_status dsa_sparse_mla_fp8_fwd(int mode, int num_q, int H, int D_qk, int D_v, float scale,
+                                  float kv_scale, const void* q, const void* kv,
+                                  long long kv_rows, const int* page_table, int max_pages,
+                                  int page_size, const int* seq_lens, const int* idx,
+                                  int k_sel, long long ld_idx, void* out, float* lse,
+                                  void* workspace, size_t workspace_bytes,
+                                  dsa_stream_t stream) {
+    g_last_error[0] = 0;
+    if (!q || !kv || !idx || !out) return fail(DSA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(out) ||
+        (lse && !aligned16(lse)))
+        return fail(DSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (num_q < 0 || H <= 0 || D_qk <= 0 || D_v <= 0 || kv_rows <= 0 || k_sel <= 0 ||
+        ld_idx < k_sel)
+        return fail(DSA_ERR_INVALID_ARG, "bad sizes");
+    if (!(scale > 0.f) || scale != scale) return fail(DSA_ERR_INVALID_ARG, "scale must be > 0");
+    if (!(kv_scale > 0.f) || !std::isfinite(kv_scale))
+        return fail(DSA_ERR_INVALID_ARG, "kv_scale must be finite and > 0");
+    if (mode != DSA_PREFILL && mode != DSA_DECODE) return fail(DSA_ERR_INVALID_ARG, "bad mode");
+    if (num_q == 0) return DSA_OK;
+    DevCtx ctx;
+    dsa_status st = check_stream_device(&ctx);
+    if (st != DSA_OK) return st;
+    return mla_absorbed(true, kv_scale, mode, num_q, H, D_qk, D_v, scale, q, kv, kv_rows,
+                        page_table, max_pages, page_size, seq_lens, idx, k_sel, ld_idx, out, lse,
+                        workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream), ctx);
+}
+
+dsa_status dsa_latent_quantize_fp8(const void* src, long long n, float kv_scale, void* dst,
+                                   dsa_stream_t stream) {
+    g_last_error[0] = 0;
+    if (n < 0) return fail(DSA_ERR_INVALID_ARG, "n must be >= 0");
+    if (n == 0) return DSA_OK;
+    if (!src || !dst) return fail(DSA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(src) || !aligned16(dst))
+        return fail(DSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (!(kv_scale > 0.f) || !std::isfinite(kv_scale))
+        return fail(DSA_ERR_INVALID_ARG, "kv_scale must be finite and > 0");
+    DevCtx ctx;
+    dsa_status st = check_stream_device(&ctx);
+    if (st != DSA_OK) return st;
+    cudaError_t e = launch_latent_quantize_fp8(static_cast<const __nv_bfloat16*>(src), n, kv_scale,
+                                               static_cast<uint8_t*>(dst),
+                                               reinterpret_cast<cudaStream_t>(stream), ctx);
+    return e == cudaSuccess ? DSA_OK : cuda_fail(e, "quantize launch");
 }
 
 size_t dsa_layer_stack_workspace_size(int T, int rows_window) {
@@ -314,10 +379,11 @@ size_t dsa_layer_stack_workspace_size(int T, int rows_window) {
     const long long ld = ((long long)T + 3) / 4 * 4;
     long long rw = rows_window;
     if (rw <= 0) {
-        // default: about 512 MB of scores per window.  Wider windows give the indexer and
-        // top-k launches enough rows to fill the GPU; at T = 65536 this is 2048 rows
-        // (the index phase measured 22.8 ms with 256-row windows, 15.9 ms with 2048).
-        rw = (512ll << 20) / (ld * 4);
+        // default: about 4 GB of scores per window.  Wider windows give the indexer and
+        // top-k launches more rows per launch and fewer launch tails: at T = 65536 this is
+        // 16384 rows, and the index phase measured 13.9 / 13.2 / 12.8 / 12.5 / 12.4 ms with
+        // 2048 / 4096 / 8192 / 16384 / 32768-row windows.
+        rw = (4096ll << 20) / (ld * 4);
         if (rw < 128) rw = 128;
     }
     if (rw > T) rw = T;

@@ -92,16 +92,22 @@ cudaError_t launch_sparse_mha_f32(const float* q, const float* k, const float* v
                                   int k_sel, long long ld_idx, float* out, float* lse,
                                   cudaStream_t stream, const DevCtx& ctx);
 
-// Absorbed-MLA sparse attention (bf16, 16 heads, 576/512) on warp-level MMAs.  Prefill
+// Absorbed-MLA sparse attention (bf16 query, 16 heads, 576/512; bf16 latent cache, or E4M3
+// codes times kv_scale when kv_fp8) on warp-level MMAs.  Prefill
 // when page_table is NULL; otherwise decode with `splits` key ranges per sequence written
 // to the partial buffers (o_part [num_q, splits, 16, 512] fp32, lse_part [num_q, splits,
 // 16]) and merged by launch_mla_combine.
-cudaError_t launch_sparse_mla_mma(const __nv_bfloat16* q, const __nv_bfloat16* kv,
-                                  long long kv_rows, const int* page_table, int max_pages,
-                                  int page_size, const int* seq_lens, const int* idx, int k_sel,
-                                  long long ld_idx, int num_q, float scale, int splits,
-                                  __nv_bfloat16* out, float* lse, float* o_part, float* lse_part,
-                                  cudaStream_t stream, const DevCtx& ctx);
+cudaError_t launch_sparse_mla_mma(const __nv_bfloat16* q, const void* kv, bool kv_fp8,
+                                  float kv_scale, long long kv_rows, const int* page_table,
+                                  int max_pages, int page_size, const int* seq_lens,
+                                  const int* idx, int k_sel, long long ld_idx, int num_q,
+                                  float scale, int splits, __nv_bfloat16* out, float* lse,
+                                  float* o_part, float* lse_part, cudaStream_t stream,
+                                  const DevCtx& ctx);
+
+// dst[i] = E4M3(src[i] / kv_scale) (round to nearest even, finite saturation).
+cudaError_t launch_latent_quantize_fp8(const __nv_bfloat16* src, long long n, float kv_scale,
+                                       uint8_t* dst, cudaStream_t stream, const DevCtx& ctx);
 
 cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int num_q, int splits,
                                __nv_bfloat16* out, float* lse, cudaStream_t stream);

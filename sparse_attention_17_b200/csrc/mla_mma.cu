@@ -37,8 +37,27 @@
 //                (exact running max shared through shared memory) and writes P in bf16.
 //                PV: warp w owns 128 of the 512 output dims (O stays in registers).
 // Two stages per CTA keep the next block's gather in flight while a block is computed.
+//
+// fp8 latent cache (DeepSeek-V2-Lite-Chat SIQ card: fp8 KV at 576 bytes per token).  The
+// same kernel, instantiated with kFp8, reads E4M3 codes (one byte per latent element,
+// value = kv_scale * code) and gathers 576-byte rows, so the shared-memory traffic per key
+// -- the bound of the bf16 kernel -- halves.  The codes are widened to f16 in registers
+// (cvt e4m3x2 -> f16x2 is exact) right after ldmatrix, and both products run as f16 warp
+// MMAs: the query is carried in f16 (exact for bf16 values of magnitude 2^-14 .. 65504)
+// and P is rounded to f16 instead of bf16.  Two tricks keep the conversion cheap:
+//   QK  the reduction over latent dims may run in any order, so an ldmatrix of fp8 rows
+//       (lane: 4 consecutive bytes of one key) feeds one m16n8k16 directly; the query
+//       fragments use the same order of dims (k = 2t,2t+1 <-> dims 4t,4t+1 and
+//       k = 2t+8,2t+9 <-> dims 4t+2,4t+3 of each 16-dim chunk).
+//   PV  ldmatrix.trans of fp8 rows gives each lane the byte pairs of two keys; one byte
+//       permute splits them into (key 2t, key 2t+1) pairs for an even and an odd dim, so
+//       one 8x8 load feeds two n-tiles, whose output dims interleave (handled at the store).
+// Four stages per CTA (the fp8 rows take half the space) keep more copies in flight.
 // Decode splits a sequence's selected keys over several units; their normalised partials
 // and log-sum-exps are merged by mla_combine_kernel.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "dsa_common.cuh"
 #include "launch.h"
 
@@ -52,13 +71,10 @@ constexpr int kDv = 512;
 constexpr int kComputeWarps = 4;
 constexpr int kBK = 32;                        // keys per block / stage
 constexpr int kCtasPerSm = 2;
-constexpr int kStages = 2;
 constexpr int kNT = kBK / 8;                   // 8-key n-tiles per block (one per compute warp)
 constexpr int kGatherWarps = kBK / 16;         // each gather warp copies 16 rows per stage
 constexpr int kGatherWarp0 = kComputeWarps;
 constexpr int kThreads = 32 * (kComputeWarps + kGatherWarps);
-constexpr int kRowPitch = 1168;                // bytes per staged key row (1152 + 16)
-constexpr int kStageBytes = kBK * kRowPitch;
 constexpr int kQPitch = 1168;                  // bytes per query head row
 constexpr int kQBytes = kH * kQPitch;          // 18688
 constexpr int kPPitch = kBK * 2 + 16;          // bytes per P row (bf16 keys + 16)
@@ -69,24 +85,42 @@ constexpr int kDvWarp = kDv / kComputeWarps;   // output dims per compute warp
 constexpr int kPVTiles = kDvWarp / 8;          // 8-dim n-tiles per compute warp
 static_assert(kNT == kComputeWarps, "each compute warp runs the softmax of one n-tile");
 static_assert(kKSteps % kComputeWarps == 0, "the K-steps split evenly over the warps");
-static_assert(kDvWarp % 16 == 0, "PV loads two n-tiles at a time");
+static_assert(kDvWarp % 32 == 0, "PV loads two n-tiles (bf16) or two 16-dim chunks (fp8) at a time");
 
+// Layout of the staged cache rows: bf16 (1152 B) or E4M3 codes (576 B) per row, padded by
+// 16 B so that the 8 rows of an ldmatrix phase hit distinct bank groups (pitch / 16 odd).
+template <bool kFp8>
+struct RowLayout {
+    static constexpr int kRowBytes = kFp8 ? kDqk : kDqk * 2;
+    static constexpr int kRowPitch = kRowBytes + 16;
+    static constexpr int kStages = kFp8 ? 4 : 2;
+    static constexpr int kStageBytes = kBK * kRowPitch;
+    static_assert((kRowPitch / 16) % 2 == 1, "row pitch must be an odd number of 16-byte units");
+    static_assert((kStages & (kStages - 1)) == 0, "stage count must be a power of two");
+};
+
+template <bool kFp8>
 struct MmaSmem {
-    alignas(128) uint8_t stage[kStages][kStageBytes];
+    using L = RowLayout<kFp8>;
+    alignas(128) uint8_t stage[L::kStages][L::kStageBytes];
     alignas(128) uint8_t q[kQBytes];
-    alignas(128) uint8_t p[kStages][kPBytes];
-    alignas(16) int valid[kStages][kBK];     // 1: the staged row holds the key; -1: not fetched
+    alignas(128) uint8_t p[L::kStages][kPBytes];
+    alignas(16) int valid[L::kStages][kBK];  // 1: the staged row holds the key; -1: not fetched
     alignas(16) float spart[kComputeWarps][kNT][32][4];  // [from warp][n-tile] partial scores
-    alignas(16) float red[kStages][kComputeWarps][kH];    // per warp, per head block maxima
+    alignas(16) float red[L::kStages][kComputeWarps][kH];  // per warp, per head block maxima
     alignas(16) float lsum[2][kComputeWarps][kH];         // per warp row sums at the end of a unit
-    uint64_t a_full[kStages], a_free[kStages];
+    uint64_t a_full[L::kStages], a_free[L::kStages];
     uint64_t q_full, q_empty;
     int abort;
 };
 
+// two CTAs per SM: each may use at most half of the SM's 228 KB less 1 KB per CTA
+static_assert(sizeof(MmaSmem<false>) + 128 <= 113 * 1024, "bf16 CTA too large for two per SM");
+static_assert(sizeof(MmaSmem<true>) + 128 <= 113 * 1024, "fp8 CTA too large for two per SM");
+
 struct Params {
     const __nv_bfloat16* q;
-    const __nv_bfloat16* kv;
+    const uint8_t* kv;       // cache rows: bf16 [.., 576] or E4M3 codes [.., 576]
     long long kv_rows;
     const int* page_table;  // NULL = prefill
     int max_pages, page_size, num_pages;
@@ -95,7 +129,8 @@ struct Params {
     int k_sel;
     long long ld_idx;
     int splits, chunk, num_units;
-    float scale_log2;
+    float scale_log2;        // softmax scale (times kv_scale for fp8) in log2 units
+    float out_scale;         // 1 (bf16) or kv_scale (fp8): multiplies the normalised output
     __nv_bfloat16* out;
     float* lse;
     float* o_part;
@@ -171,6 +206,33 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// The same with f16 operands (the fp8 cache path).
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                        uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Two E4M3 codes (low / high byte of the low 16 bits) -> f16x2 (low / high half); exact.
+__device__ __forceinline__ uint32_t e4m3x2_lo_to_f16x2(uint32_t v) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(v & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+__device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2(uint32_t v) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(v >> 16), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+// bf16x2 -> f16x2 (round to nearest; exact for magnitudes 2^-14 .. 65504).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -185,10 +247,16 @@ __device__ __forceinline__ void wait_soft(uint64_t* bar, uint32_t parity, volati
     (void)mbar_wait(bar, parity, abort, err);
 }
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 sparse_mla_mma_kernel(const Params p) {
+    using L = RowLayout<kFp8>;
+    constexpr int kStages = L::kStages;
+    constexpr int kRowPitch = L::kRowPitch;
+    constexpr int kRowBytes = L::kRowBytes;
     extern __shared__ uint8_t smem_raw[];
-    MmaSmem& sm = *reinterpret_cast<MmaSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    MmaSmem<kFp8>& sm =
+        *reinterpret_cast<MmaSmem<kFp8>*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     volatile int* abort = &sm.abort;
@@ -236,31 +304,31 @@ sparse_mla_mma_kernel(const Params p) {
             int s_ahead = lane < 16 ? load_index(p, x, e_lane + kBK) : -1;
             long long row_next = lane < 16 ? resolve_row(p, x, load_index(p, x, e_lane)) : -1;
             for (int j = 0; j < x.nb; ++j, ++G) {
-                const int s = G & 1;
+                const int s = G % kStages;
                 const long long row = row_next;
                 if (lane < 16) {
                     const int s_far = load_index(p, x, e_lane + (j + 2) * kBK);
                     row_next = resolve_row(p, x, s_ahead);
                     s_ahead = s_far;
                 }
-                wait_soft(&sm.a_free[s], ((G >> 1) & 1) ^ 1, abort, p.err);
+                wait_soft(&sm.a_free[s], ((G / kStages) & 1) ^ 1, abort, p.err);
                 if (lane < 16) sm.valid[s][gw * 16 + lane] = row >= 0 ? 1 : -1;
                 const unsigned vmask = __ballot_sync(0xffffffffu, row >= 0);
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive_expect_tx(&sm.a_full[s], (uint32_t)__popc(vmask) * (kDqk * 2));
+                    mbar_arrive_expect_tx(&sm.a_full[s], (uint32_t)__popc(vmask) * kRowBytes);
                 __syncwarp();
                 if (row >= 0)
-                    bulk_load(sm.stage[s] + (gw * 16 + lane) * kRowPitch, p.kv + row * kDqk,
-                              kDqk * 2, &sm.a_full[s]);
+                    bulk_load(sm.stage[s] + (gw * 16 + lane) * kRowPitch, p.kv + row * kRowBytes,
+                              kRowBytes, &sm.a_full[s]);
             }
         }
         // The compute warps consume every block and query, but after a timed-out wait they
         // may not have: let the last copies land (time-bounded, whatever the abort flag
         // says) before the CTA can exit.
         volatile int keep_waiting = 0;
-        for (uint32_t Gl = G >= 2 ? G - 2 : 0; Gl < G; ++Gl)
-            (void)mbar_wait(&sm.a_full[Gl & 1], (Gl >> 1) & 1, &keep_waiting, p.err);
+        for (uint32_t Gl = G >= kStages ? G - kStages : 0; Gl < G; ++Gl)
+            (void)mbar_wait(&sm.a_full[Gl % kStages], (Gl / kStages) & 1, &keep_waiting, p.err);
         if (leader && units > 0) (void)mbar_wait(&sm.q_full, (units - 1) & 1, &keep_waiting, p.err);
     } else {
         // ================================ compute ===============================
@@ -275,12 +343,24 @@ sparse_mla_mma_kernel(const Params p) {
             const Unit x = unit_of(p, u);
             wait_soft(&sm.q_full, ui & 1, abort, p.err);
             uint32_t qa[kKQuarter][4];
-            {
+            if constexpr (!kFp8) {
                 const int head = (lane & 7) + ((lane >> 3) & 1) * 8;
                 const uint32_t qrow = smem_u32(sm.q) + head * kQPitch + ((lane >> 4) & 1) * 16;
 #pragma unroll
                 for (int ks = 0; ks < kKQuarter; ++ks)
                     ldsm_x4(qrow + (warp * kKQuarter + ks) * 32, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+            } else {
+                // f16 fragments in the permuted order of dims of the fp8 QK (see the top)
+#pragma unroll
+                for (int ks = 0; ks < kKQuarter; ++ks) {
+                    const int d0 = (warp * kKQuarter + ks) * 16 + 4 * t;
+                    const uint2 lo = *reinterpret_cast<const uint2*>(sm.q + g * kQPitch + d0 * 2);
+                    const uint2 hi = *reinterpret_cast<const uint2*>(sm.q + (g + 8) * kQPitch + d0 * 2);
+                    qa[ks][0] = bf16x2_to_f16x2(lo.x);
+                    qa[ks][1] = bf16x2_to_f16x2(hi.x);
+                    qa[ks][2] = bf16x2_to_f16x2(lo.y);
+                    qa[ks][3] = bf16x2_to_f16x2(hi.y);
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.q_empty);
@@ -292,14 +372,14 @@ sparse_mla_mma_kernel(const Params p) {
             float l_lse[2] = {0.f, 0.f};              // the same before bf16 rounding
 
             for (int j = 0; j < x.nb; ++j, ++G) {
-                const int s = G & 1;
-                wait_soft(&sm.a_full[s], (G >> 1) & 1, abort, p.err);
+                const int s = G % kStages;
+                wait_soft(&sm.a_full[s], (G / kStages) & 1, abort, p.err);
                 const uint32_t st = smem_u32(sm.stage[s]);
                 // ---- QK: S[16 heads x kBK keys] over this warp's K-quarter ----
                 float acc[kNT][4];
 #pragma unroll
                 for (int i = 0; i < kNT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-                {
+                if constexpr (!kFp8) {
                     const int key = (lane & 7) + ((lane >> 4) & 1) * 8;
                     const uint32_t krow = st + key * kRowPitch + ((lane >> 3) & 1) * 16 + warp * kKQuarter * 32;
 #pragma unroll
@@ -311,6 +391,18 @@ sparse_mla_mma_kernel(const Params p) {
                             mma_bf16(acc[2 * n2], qa[ks], b0, b1);
                             mma_bf16(acc[2 * n2 + 1], qa[ks], b2, b3);
                         }
+                    }
+                } else {
+                    // one x4 load = the 16 code bytes of this K-step for all 32 keys; matrix
+                    // j (lanes 8j..8j+7 address keys 8j..8j+7) is n-tile j
+                    const uint32_t krow = st + lane * kRowPitch + warp * kKQuarter * 16;
+#pragma unroll
+                    for (int ks = 0; ks < kKQuarter; ++ks) {
+                        uint32_t r[4];
+                        ldsm_x4(krow + ks * 16, r[0], r[1], r[2], r[3]);
+#pragma unroll
+                        for (int nt = 0; nt < kNT; ++nt)
+                            mma_f16(acc[nt], qa[ks], e4m3x2_lo_to_f16x2(r[nt]), e4m3x2_hi_to_f16x2(r[nt]));
                     }
                 }
                 // partial sums of the other warps' n-tiles go through shared memory
@@ -367,9 +459,16 @@ sparse_mla_mma_kernel(const Params p) {
                 for (int r = 0; r < 2; ++r) {
                     const float p0 = exp2f(sc[2 * r] - ref[r]);
                     const float p1 = exp2f(sc[2 * r + 1] - ref[r]);
-                    const uint32_t pk = pack_bf16(p0, p1);
-                    const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&pk);
-                    l_run[r] += __bfloat162float(pr.x) + __bfloat162float(pr.y);
+                    uint32_t pk;
+                    if constexpr (!kFp8) {
+                        pk = pack_bf16(p0, p1);
+                        const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&pk);
+                        l_run[r] += __bfloat162float(pr.x) + __bfloat162float(pr.y);
+                    } else {
+                        pk = pack_f16(p0, p1);
+                        const __half2 pr = *reinterpret_cast<const __half2*>(&pk);
+                        l_run[r] += __low2float(pr) + __high2float(pr);
+                    }
                     l_lse[r] += p0 + p1;
                     *reinterpret_cast<uint32_t*>(sm.p[s] + (g + 8 * r) * kPPitch + (warp * 8 + 2 * t) * 2) = pk;
                 }
@@ -384,17 +483,43 @@ sparse_mla_mma_kernel(const Params p) {
                     const int head = (lane & 7) + ((lane >> 3) & 1) * 8;
                     const uint32_t prow = smem_u32(sm.p[s]) + head * kPPitch + ((lane >> 4) & 1) * 16;
                     const int vkey = (lane & 7) + ((lane >> 3) & 1) * 8;
-                    const uint32_t vrow = st + vkey * kRowPitch + (warp * kDvWarp + ((lane >> 4) & 1) * 8) * 2;
+                    if constexpr (!kFp8) {
+                        const uint32_t vrow = st + vkey * kRowPitch + (warp * kDvWarp + ((lane >> 4) & 1) * 8) * 2;
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-                        uint32_t pa[4];
-                        ldsm_x4(prow + kk * 32, pa[0], pa[1], pa[2], pa[3]);
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
+                            uint32_t pa[4];
+                            ldsm_x4(prow + kk * 32, pa[0], pa[1], pa[2], pa[3]);
 #pragma unroll
-                        for (int n2 = 0; n2 < kPVTiles / 2; ++n2) {
-                            uint32_t b0, b1, b2, b3;
-                            ldsm_x4_t(vrow + kk * 16 * kRowPitch + n2 * 32, b0, b1, b2, b3);
-                            mma_bf16(o[2 * n2], pa, b0, b1);
-                            mma_bf16(o[2 * n2 + 1], pa, b2, b3);
+                            for (int n2 = 0; n2 < kPVTiles / 2; ++n2) {
+                                uint32_t b0, b1, b2, b3;
+                                ldsm_x4_t(vrow + kk * 16 * kRowPitch + n2 * 32, b0, b1, b2, b3);
+                                mma_bf16(o[2 * n2], pa, b0, b1);
+                                mma_bf16(o[2 * n2 + 1], pa, b2, b3);
+                            }
+                        }
+                    } else {
+                        // x4.trans: matrices (keys 0-7 | 8-15) x (chunk c | c+1) of 16 dims;
+                        // lane (g,t) gets bytes [V(2t,2g) V(2t,2g+1) V(2t+1,2g) V(2t+1,2g+1)]
+                        // of its chunk; the byte permute 3120 pairs them per dim.  n-tile
+                        // 4*c2 + 2*(c&1) holds the even dims of chunk c, the next tile the
+                        // odd dims.
+                        const uint32_t vrow = st + vkey * kRowPitch + warp * kDvWarp + ((lane >> 4) & 1) * 16;
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
+                            uint32_t pa[4];
+                            ldsm_x4(prow + kk * 32, pa[0], pa[1], pa[2], pa[3]);
+#pragma unroll
+                            for (int c2 = 0; c2 < kPVTiles / 4; ++c2) {
+                                uint32_t r[4];
+                                ldsm_x4_t(vrow + kk * 16 * kRowPitch + c2 * 32, r[0], r[1], r[2], r[3]);
+#pragma unroll
+                                for (int h = 0; h < 2; ++h) {
+                                    const uint32_t x0 = __byte_perm(r[2 * h], 0u, 0x3120);
+                                    const uint32_t x1 = __byte_perm(r[2 * h + 1], 0u, 0x3120);
+                                    mma_f16(o[4 * c2 + 2 * h], pa, e4m3x2_lo_to_f16x2(x0), e4m3x2_lo_to_f16x2(x1));
+                                    mma_f16(o[4 * c2 + 2 * h + 1], pa, e4m3x2_hi_to_f16x2(x0), e4m3x2_hi_to_f16x2(x1));
+                                }
+                            }
                         }
                     }
                 }
@@ -425,10 +550,32 @@ sparse_mla_mma_kernel(const Params p) {
                 Lx[0] += sm.lsum[1][i][g];
                 Lx[1] += sm.lsum[1][i][g + 8];
             }
-            const float inv0 = (x.nb > 0 && L[0] > 0.f) ? 1.f / L[0] : 0.f;
-            const float inv1 = (x.nb > 0 && L[1] > 0.f) ? 1.f / L[1] : 0.f;
+            const float inv0 = (x.nb > 0 && L[0] > 0.f) ? p.out_scale / L[0] : 0.f;
+            const float inv1 = (x.nb > 0 && L[1] > 0.f) ? p.out_scale / L[1] : 0.f;
+            if constexpr (kFp8) {
+                // chunk c of this warp: dims 16c + 4t + {0,1,2,3} are (even tile, odd tile)
+                // x (column 0, column 1) -- see the PV comment
 #pragma unroll
-            for (int n = 0; n < kPVTiles; ++n) {
+                for (int c = 0; c < kPVTiles / 2; ++c) {
+                    const int te = 4 * (c >> 1) + 2 * (c & 1);
+                    const int dim = warp * kDvWarp + 16 * c + 4 * t;
+                    const float v0[4] = {o[te][0] * inv0, o[te + 1][0] * inv0, o[te][1] * inv0, o[te + 1][1] * inv0};
+                    const float v1[4] = {o[te][2] * inv1, o[te + 1][2] * inv1, o[te][3] * inv1, o[te + 1][3] * inv1};
+                    if (p.page_table == nullptr) {
+                        __nv_bfloat16* o0 = p.out + ((long long)x.n * kH + g) * kDv + dim;
+                        __nv_bfloat16* o1 = p.out + ((long long)x.n * kH + g + 8) * kDv + dim;
+                        *reinterpret_cast<uint2*>(o0) = make_uint2(pack_bf16(v0[0], v0[1]), pack_bf16(v0[2], v0[3]));
+                        *reinterpret_cast<uint2*>(o1) = make_uint2(pack_bf16(v1[0], v1[1]), pack_bf16(v1[2], v1[3]));
+                    } else {
+                        float* o0 = p.o_part + (((long long)x.n * p.splits + x.sp) * kH + g) * kDv + dim;
+                        float* o1 = p.o_part + (((long long)x.n * p.splits + x.sp) * kH + g + 8) * kDv + dim;
+                        *reinterpret_cast<float4*>(o0) = make_float4(v0[0], v0[1], v0[2], v0[3]);
+                        *reinterpret_cast<float4*>(o1) = make_float4(v1[0], v1[1], v1[2], v1[3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < (kFp8 ? 0 : kPVTiles); ++n) {
                 const int dim = warp * kDvWarp + n * 8 + 2 * t;
                 if (p.page_table == nullptr) {
                     __nv_bfloat16* o0 = p.out + ((long long)x.n * kH + g) * kDv + dim;
@@ -519,17 +666,40 @@ int mla_decode_splits(int num_q, int k_sel, int num_sms) {
     return best;
 }
 
-size_t mla_mma_smem_bytes() { return sizeof(MmaSmem) + 128; }
+size_t mla_mma_smem_bytes(bool fp8) {
+    return (fp8 ? sizeof(MmaSmem<true>) : sizeof(MmaSmem<false>)) + 128;
+}
 
-cudaError_t launch_sparse_mla_mma(const __nv_bfloat16* q, const __nv_bfloat16* kv,
-                                  long long kv_rows, const int* page_table, int max_pages,
-                                  int page_size, const int* seq_lens, const int* idx, int k_sel,
-                                  long long ld_idx, int num_q, float scale, int splits,
-                                  __nv_bfloat16* out, float* lse, float* o_part, float* lse_part,
-                                  cudaStream_t stream, const DevCtx& ctx) {
+namespace {
+template <bool kFp8>
+cudaError_t launch_mla_kernel(const Params& p, cudaStream_t stream, const DevCtx& ctx) {
+    const size_t smem = mla_mma_smem_bytes(kFp8);
+    cudaError_t e = cudaFuncSetAttribute(sparse_mla_mma_kernel<kFp8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // two CTAs per SM need most of the shared memory carve-out
+    e = cudaFuncSetAttribute(sparse_mla_mma_kernel<kFp8>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    const int slots = kCtasPerSm * ctx.num_sms;
+    const int grid = p.num_units < slots ? p.num_units : slots;
+    sparse_mla_mma_kernel<kFp8><<<grid, kThreads, smem, stream>>>(p);
+    count_launch(DSA_KERNEL_ATTENTION);
+    return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_sparse_mla_mma(const __nv_bfloat16* q, const void* kv, bool kv_fp8,
+                                  float kv_scale, long long kv_rows, const int* page_table,
+                                  int max_pages, int page_size, const int* seq_lens,
+                                  const int* idx, int k_sel, long long ld_idx, int num_q,
+                                  float scale, int splits, __nv_bfloat16* out, float* lse,
+                                  float* o_part, float* lse_part, cudaStream_t stream,
+                                  const DevCtx& ctx) {
     Params p{};
     p.q = q;
-    p.kv = kv;
+    p.kv = static_cast<const uint8_t*>(kv);
     p.kv_rows = kv_rows;
     p.page_table = page_table;
     p.max_pages = max_pages;
@@ -542,25 +712,14 @@ cudaError_t launch_sparse_mla_mma(const __nv_bfloat16* q, const __nv_bfloat16* k
     p.splits = page_table ? splits : 1;
     p.chunk = page_table ? ((k_sel + splits - 1) / splits + kBK - 1) / kBK * kBK : k_sel;
     p.num_units = num_q * p.splits;
-    p.scale_log2 = scale * 1.4426950408889634f;
+    p.scale_log2 = scale * (kv_fp8 ? kv_scale : 1.f) * 1.4426950408889634f;
+    p.out_scale = kv_fp8 ? kv_scale : 1.f;
     p.out = out;
     p.lse = lse;
     p.o_part = o_part;
     p.lse_part = lse_part;
     p.err = ctx.err;
-    const size_t smem = mla_mma_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(sparse_mla_mma_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    // two CTAs per SM need most of the shared memory carve-out
-    e = cudaFuncSetAttribute(sparse_mla_mma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             (int)cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    const int slots = kCtasPerSm * ctx.num_sms;
-    const int grid = p.num_units < slots ? p.num_units : slots;
-    sparse_mla_mma_kernel<<<grid, kThreads, smem, stream>>>(p);
-    count_launch(DSA_KERNEL_ATTENTION);
-    return cudaGetLastError();
+    return kv_fp8 ? launch_mla_kernel<true>(p, stream, ctx) : launch_mla_kernel<false>(p, stream, ctx);
 }
 
 cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int num_q, int splits,

@@ -87,8 +87,7 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     // every (sequence, split) unit overwrites its partial output and log-sum-exp, so the
     // array needs no clearing between calls
-    e = launch_sparse_mla_mma(static_cast<const __nv_bfloat16*>(q),
-                               static_cast<const __nv_bfloat16*>(kv), kv_rows, page_table,
+    e = launch_sparse_mla_mma(static_cast<const __nv_bfloat16*>(q), kv, false, 1.f, kv_rows, page_table,
                                max_pages, page_size, seq_lens, idx, k_sel, ld_idx, num_q, scale,
                                splits, nullptr, nullptr, o_part, lse_part, cs, ctx);
     if (e != cudaSuccess) return DSA_ERR_CUDA;

@@ -130,18 +130,45 @@ def test_attention_rejects(lib):
              None, None, 0, None) == _lib.DSA_OK
 
 
+def test_fp8_attention_and_quantize_reject(lib):
+    f = lib.dsa_sparse_mla_fp8_fwd
+    ok = (0, 4, 16, 576, 512, 0.1, 0.01, 16, 16, 8, None, 0, 0, None, 16, 4, 4, 16, None, None,
+          0, None)
+    # kv_scale must be finite and positive
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        a = list(ok)
+        a[6] = bad
+        assert f(*a) == _lib.DSA_ERR_INVALID_ARG and "kv_scale" in lib.dsa_last_error().decode()
+    a = list(ok)
+    a[7] = None  # null q
+    assert f(*a) == _lib.DSA_ERR_INVALID_ARG
+    a = list(ok)
+    a[1] = 0  # empty batch: no-op before any device work
+    assert f(*a) == _lib.DSA_OK
+    # the bf16 entry point refuses an fp8 dtype (no scale to apply)
+    g = lib.dsa_sparse_mla_fwd
+    assert g(2, 0, 4, 16, 1, 576, 512, 0.1, 16, 16, None, 8, None, 0, 0, None, 16, 4, 4, 16,
+             None, None, 0, None) == _lib.DSA_ERR_INVALID_ARG
+    q = lib.dsa_latent_quantize_fp8
+    assert q(16, 0, 0.01, 16, None) == _lib.DSA_OK
+    assert q(16, -1, 0.01, 16, None) == _lib.DSA_ERR_INVALID_ARG
+    assert q(None, 8, 0.01, 16, None) == _lib.DSA_ERR_INVALID_ARG
+    assert q(18, 8, 0.01, 16, None) == _lib.DSA_ERR_INVALID_ARG
+    assert q(16, 8, 0.0, 16, None) == _lib.DSA_ERR_INVALID_ARG
+
+
 def test_workspace_sizes(lib):
     assert lib.dsa_sparse_mla_workspace_size(0, 100, 16, 512, 2048) == 0
     ws = lib.dsa_sparse_mla_workspace_size(1, 64, 16, 512, 2048)
     assert ws > 0 and ws % (64 * 16 * 513 * 4) == 0
-    assert lib.dsa_layer_stack_workspace_size(65536, 0) == 512 << 20
+    assert lib.dsa_layer_stack_workspace_size(65536, 0) == 4096 << 20
     assert lib.dsa_layer_stack_workspace_size(1000, 0) == 1000 * 1000 * 4
     assert lib.dsa_layer_stack_workspace_size(100, 16) == 16 * 100 * 4
 
 
 def test_launch_counters_reset(lib):
     dsa.reset_launch_counts()
-    for k in range(4):
+    for k in range(5):
         assert dsa.launch_count(k) == 0
     assert dsa.launch_count(9) == -1
 
