@@ -109,6 +109,8 @@ def load_peaks():
 
 
 def kernel_source_hash(name):
+    """Hash of a kernel's source file (name, or name:variant) and the shared header."""
+    name = name.split(":")[0]
     h = hashlib.sha256()
     for f in sorted((ROOT / "sparse_attention_17_b200" / "csrc").glob("*")):
         if f.name in (name, "dsa_common.cuh"):

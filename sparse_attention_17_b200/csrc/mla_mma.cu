@@ -56,7 +56,6 @@
 // Decode splits a sequence's selected keys over several units; their normalised partials
 // and log-sum-exps are merged by mla_combine_kernel.
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 
 #include "dsa_common.cuh"
 #include "launch.h"
@@ -215,14 +214,19 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-// Two E4M3 codes (low / high byte of the low 16 bits) -> f16x2 (low / high half); exact.
+// Two E4M3 codes (bytes 0,1 or bytes 2,3 of v) -> f16x2 (low byte -> low half); exact.
+// One cvt on a half of the register, with no repacking of the result.
 __device__ __forceinline__ uint32_t e4m3x2_lo_to_f16x2(uint32_t v) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(v & 0xffffu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
+        : "=r"(r) : "r"(v));
+    return r;
 }
 __device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2(uint32_t v) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(v >> 16), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, hi;\n\t}"
+        : "=r"(r) : "r"(v));
+    return r;
 }
 // bf16x2 -> f16x2 (round to nearest; exact for magnitudes 2^-14 .. 65504).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
