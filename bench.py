@@ -39,9 +39,11 @@ def parse_args(argv=None):
     ap.add_argument("--topk", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--workload", choices=["prefill", "decode", "stack"], default="prefill",
+    ap.add_argument("--workload", choices=["prefill", "decode", "stack", "varlen"],
+                    default="prefill",
                     help="prefill: the T=65536 headline; decode: 64 sequences x 32768 paged "
-                         "tokens; stack: the 27-layer FSS x 9 IndexCache stack at T=16384")
+                         "tokens; stack: the 27-layer FSS x 9 IndexCache stack at T=16384; "
+                         "varlen: 16 packed prompts of 512..8192 tokens in one batch")
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
                     help="latent cache: bf16, or E4M3 codes times one fp32 scale")
     ap.add_argument("--window-rows", type=int, default=0,
@@ -506,6 +508,50 @@ def run_decode(args, local_rank):
                         "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": src}}
 
 
+def run_varlen(args, local_rank):
+    """Batched prefill of 16 independent prompts with lengths drawn uniformly from
+    512..8192 tokens, packed along the token axis: dsa_index_varlen (indexer + top-k per
+    sequence) and one sparse MLA over the packed batch."""
+    import numpy as np
+    import torch
+    import sparse_attention_17_b200 as dsa
+    from sparse_attention_17_b200 import inputs as G
+    torch.cuda.set_device(local_rank)
+    k = args.topk
+    lens = [int(v) for v in np.random.default_rng(0).integers(512, 8193, 16)]
+    starts = [int(v) for v in np.cumsum([0] + lens[:-1])]
+    N = sum(lens)
+    host = G.mla_prefill_gauss(T=N, seed=0, k=k)
+    x = {n: host[n].cuda() for n in ("q_idx", "k_idx", "w", "q", "kv")}
+    idx = torch.empty((N, k), dtype=torch.int32, device="cuda")
+    out = torch.empty((N, 16, 512), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(dsa.index_varlen_workspace_size(max(lens), args.window_rows) // 4,
+                     device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def index():
+        dsa.index_varlen(x["q_idx"], x["k_idx"], x["w"], starts, lens, k, idx, ws)
+
+    def mla():
+        dsa.sparse_mla_fwd(x["q"], x["kv"], idx, out, G.SCALE_MLA)
+
+    def step():
+        index(); mla()
+
+    ms = _timed(step, args.steps, args.warmup, stream)
+    t_idx = _timed(index, args.steps, 1, stream)
+    t_mla = _timed(mla, args.steps, 1, stream)
+    assert dsa.check_device_errors() == 0
+    return {"metric": "DSA batched prefill tokens/sec (16 packed prompts, 512..8192 tokens, "
+                      "top-2048)", "value": round(N / (ms / 1e3), 1), "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "dsa_varlen_prefill_16seq_top2048", "tokens": N,
+                       "seq_lens": lens},
+            "kernels": {"index_varlen_ms": round(t_idx, 4), "sparse_mla_ms": round(t_mla, 4)}}
+
+
 def run_stack(args, local_rank):
     """The IndexCache stack: 27 layers "FSS" x 9 at T=16384, top-2048, through
     dsa_layer_stack (9 indexer + top-k passes, 27 sparse MLA passes)."""
@@ -593,6 +639,8 @@ def main(argv=None):
             res = run_decode(args, local_rank) if rank == 0 else None
         elif args.workload == "stack":
             res = run_stack(args, local_rank) if rank == 0 else None
+        elif args.workload == "varlen":
+            res = run_varlen(args, local_rank) if rank == 0 else None
         else:
             res = run_native(args, rank, world, local_rank)
     finally:

@@ -232,6 +232,36 @@ dsa_status dsa_sparse_mla_decode_noalloc(int num_q, int H, int D_qk, int D_v, fl
                                          dsa_stream_t stream);
 
 /*
+ * dsa_index_varlen -- indexer + top-k for a batch of independent prefill sequences packed
+ * along the token axis (batched prefill of unequal lengths; a left-padded batch [B, T] is
+ * the packing with sequence b at rows b*T + pad_b .. (b+1)*T - 1 and the pads outside
+ * every sequence).  DSV2-Lite-IndexCache card: causal selection per query, and batched
+ * generation with left padding.
+ *
+ * Sequence b holds the tokens seq_start[b] .. seq_start[b] + seq_len[b] - 1 of
+ *   q_idx [num_tokens, 16, 64] bf16, k_idx [num_tokens, 64] bf16, w [num_tokens, 16] fp32.
+ * Token t of sequence b selects, exactly as dsa_indexer_scores + dsa_topk_select would for
+ * that sequence alone, the top-k of I(t, s) over its own keys s = seq_start[b] .. t.
+ * idx [num_tokens, ld_idx] int32: row t receives the selected keys as PACKED token rows
+ * (so that dsa_sparse_mla_fwd in prefill mode reads them from the packed latent cache),
+ * ascending, -1 padded.  Rows outside every sequence are not written.
+ * seq_start, seq_len: HOST int32 arrays of num_seqs entries; sequences lie inside
+ * [0, num_tokens), in increasing order, without overlap; lengths 0 .. 262144.
+ * workspace: device memory for score rows, at least dsa_index_varlen_workspace_size(
+ * longest sequence, 1) bytes; a larger workspace scores more rows per launch.
+ * Launches one indexer and one top-k per sequence and window of rows; nothing is
+ * synchronised.  Errors: as for dsa_indexer_scores / dsa_topk_select.
+ */
+dsa_status dsa_index_varlen(const void* q_idx, const void* k_idx, const float* w, int H_I,
+                            int D_I, int num_tokens, int num_seqs, const int* seq_start,
+                            const int* seq_len, int k, int* idx, long long ld_idx,
+                            void* workspace, size_t workspace_bytes, dsa_stream_t stream);
+
+/* Workspace bytes for dsa_index_varlen with windows of rows_window rows of the longest
+ * sequence (0 = the library's default window, about 4 GB of scores). */
+size_t dsa_index_varlen_workspace_size(int max_seq_len, int rows_window);
+
+/*
  * dsa_sparse_mla_fp8_fwd -- dsa_sparse_mla_fwd (absorbed MLA, bf16 query, prefill or paged
  * decode) over an fp8 latent cache.  DeepSeek-V2-Lite-Chat SIQ card (what is quantized,
  * KV-cache bullet): fp8 KV at 576 bytes per token, one byte per latent element.

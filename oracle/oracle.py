@@ -216,6 +216,26 @@ def prefill_indices(q_idx, k_idx, w, k: int, q_begin: int = 0, rows: int | None 
     return topk(sc, causal_n_valid(q_begin, rows), k, mutant=mutant)
 
 
+def prefill_indices_varlen(q_idx, k_idx, w, seq_start, seq_len, k: int, fill: int = -1,
+                           mutant: int = 0) -> np.ndarray:
+    """Batched prefill of packed sequences (DSV2-Lite-IndexCache card: causal selection per
+    query; batched generation with left padding).  Sequence b is an independent prompt
+    over the tokens seq_start[b] .. seq_start[b]+seq_len[b]-1: its queries select among
+    its own earlier keys only.  Indices are returned as packed token rows; rows outside
+    every sequence hold `fill`.  (Mutant 13: the packed offset is left off.)"""
+    N = q_idx.shape[0]
+    out = np.full((N, k), fill, dtype=np.int32)
+    for s0, L in zip(seq_start, seq_len):
+        s0, L = int(s0), int(L)
+        if L == 0:
+            continue
+        sl = slice(s0, s0 + L)
+        idx = prefill_indices(q_idx[sl], k_idx[sl], w[sl], k, mutant=mutant)
+        off = 0 if mutant == 13 else s0
+        out[sl] = np.where(idx >= 0, idx + off, -1)
+    return out
+
+
 def layer_stack(pattern: str, layers: list[dict], k: int, scale: float, d_v: int = 512,
                 mutant: int = 0):
     """IndexCache layer loop (vLLM IndexCache docs, "How It Works"): an 'F' layer computes
@@ -260,7 +280,8 @@ def pattern_from_freq(freq: int, num_layers: int) -> str:
 # with exponent and mantissa fields all ones (0x7f / 0xff) is NaN; there is no infinity,
 # so the largest finite magnitude is 1.75 * 2^8 = 448.
 #
-# Mutants 9..12 (Python-side planted mistakes for the pin mutation test):
+# Mutants 9..12 (Python-side planted mistakes for the pin mutation test; 13 is in
+# prefill_indices_varlen):
 #   9  exponent bias 8 instead of 7        10  subnormals decoded as normals
 #   11 encoder ties rounded away from zero 12  kv_scale left off the attention output
 def e4m3_decode(codes, mutant: int = 0) -> np.ndarray:

@@ -40,6 +40,8 @@ SYMBOLS = [
     ("dsa_sparse_mla_workspace_size", _SZ, [_I, _I, _I, _I, _I]),
     ("dsa_sparse_mla_decode_noalloc", _I, [_I, _I, _I, _I, _F, _P, _P, _LL, _P, _I, _I, _P, _P, _I,
                                            _LL, _P, _P, _P]),
+    ("dsa_index_varlen", _I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _LL, _P, _SZ, _P]),
+    ("dsa_index_varlen_workspace_size", _SZ, [_I, _I]),
     ("dsa_sparse_mla_fp8_fwd", _I, [_I, _I, _I, _I, _I, _F, _F, _P, _P, _LL, _P, _I, _I, _P, _P,
                                     _I, _LL, _P, _P, _P, _SZ, _P]),
     ("dsa_latent_quantize_fp8", _I, [_P, _LL, _F, _P, _P]),
@@ -276,6 +278,31 @@ def sparse_mla_fp8_fwd(q, kv, kv_scale: float, idx, out, scale: float, lse=None,
                                           seq_lens.data_ptr(), idx.data_ptr(), k_sel,
                                           idx.stride(0), out.data_ptr(), _ptr(lse), ws_ptr,
                                           ws_bytes, _stream()))
+
+
+def index_varlen_workspace_size(max_seq_len: int, rows_window: int = 0) -> int:
+    return load().dsa_index_varlen_workspace_size(max_seq_len, rows_window)
+
+
+def index_varlen(q_idx, k_idx, w, seq_start, seq_len, k: int, idx, workspace) -> None:
+    """dsa_index_varlen: packed sequences (host lists seq_start / seq_len) of q_idx
+    [N,16,64], k_idx [N,64], w [N,16]; idx [N, >=k] receives packed-row indices."""
+    lib = load()
+    _need(q_idx, torch.bfloat16, 3, "q_idx")
+    _need(k_idx, torch.bfloat16, 2, "k_idx")
+    _need(w, torch.float32, 2, "w")
+    _need(idx, torch.int32, 2, "idx")
+    n = len(seq_start)
+    if len(seq_len) != n:
+        raise ValueError("seq_start and seq_len must have the same length")
+    arr = ctypes.c_int * max(n, 1)
+    starts, lens = arr(*[int(v) for v in seq_start]), arr(*[int(v) for v in seq_len])
+    _check(lib.dsa_index_varlen(q_idx.data_ptr(), k_idx.data_ptr(), w.data_ptr(), q_idx.shape[1],
+                                q_idx.shape[2], q_idx.shape[0], n,
+                                ctypes.cast(starts, ctypes.c_void_p),
+                                ctypes.cast(lens, ctypes.c_void_p), k, idx.data_ptr(),
+                                idx.stride(0), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), _stream()))
 
 
 def latent_quantize_fp8(src, kv_scale: float, dst) -> None:

@@ -374,6 +374,79 @@ dsa_status dsa_latent_quantize_fp8(const void* src, long long n, float kv_scale,
     return e == cudaSuccess ? DSA_OK : cuda_fail(e, "quantize launch");
 }
 
+size_t dsa_index_varlen_workspace_size(int max_seq_len, int rows_window) {
+    if (max_seq_len <= 0) return 0;
+    const long long ld = ((long long)max_seq_len + 3) / 4 * 4;
+    long long rw = rows_window > 0 ? rows_window : dsa_layer_stack_workspace_size(max_seq_len, 0) / (ld * 4);
+    if (rw > max_seq_len) rw = max_seq_len;
+    if (rw < 1) rw = 1;
+    return (size_t)(rw * ld * 4);
+}
+
+dsa_status dsa_index_varlen(const void* q_idx, const void* k_idx, const float* w, int H_I, int D_I,
+                            int num_tokens, int num_seqs, const int* seq_start, const int* seq_len,
+                            int k, int* idx, long long ld_idx, void* workspace,
+                            size_t workspace_bytes, dsa_stream_t stream) {
+    g_last_error[0] = 0;
+    if (num_seqs < 0 || num_tokens < 0) return fail(DSA_ERR_INVALID_ARG, "negative sizes");
+    if (num_seqs == 0) return DSA_OK;
+    if (!seq_start || !seq_len) return fail(DSA_ERR_INVALID_ARG, "seq_start / seq_len missing");
+    if (!q_idx || !k_idx || !w || !idx) return fail(DSA_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(idx))
+        return fail(DSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (H_I != 16 || D_I != 64)
+        return fail(DSA_ERR_UNSUPPORTED, "bf16 indexer supports H_I=16, D_I=64 only");
+    if (k < 1 || k > 4096) return fail(DSA_ERR_UNSUPPORTED, "k must be in [1, 4096]");
+    if (ld_idx < k) return fail(DSA_ERR_INVALID_ARG, "ld_idx < k");
+    // the sequences: inside [0, num_tokens), in increasing order, not overlapping
+    int max_len = 0;
+    long long prev_end = 0;
+    for (int b = 0; b < num_seqs; ++b) {
+        const long long s0 = seq_start[b], L = seq_len[b];
+        if (s0 < 0 || L < 0 || s0 + L > num_tokens)
+            return fail(DSA_ERR_INVALID_ARG, "sequence %d [%lld, %lld) outside [0, %d)", b, s0,
+                        s0 + L, num_tokens);
+        if (s0 < prev_end)
+            return fail(DSA_ERR_INVALID_ARG, "sequence %d starts before the end of the previous one", b);
+        if (L > 262144) return fail(DSA_ERR_UNSUPPORTED, "sequences of at most 262144 tokens");
+        prev_end = s0 + L;
+        if (L > max_len) max_len = (int)L;
+    }
+    if (max_len == 0) return DSA_OK;
+    const long long ld = ((long long)max_len + 3) / 4 * 4;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < (size_t)(ld * 4))
+        return fail(DSA_ERR_WORKSPACE, "workspace must hold at least one row of %lld scores", ld);
+    const long long rw = (long long)(workspace_bytes / (ld * 4));
+    DevCtx ctx;
+    dsa_status st = check_stream_device(&ctx);
+    if (st != DSA_OK) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    float* scores = static_cast<float*>(workspace);
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q_idx);
+    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k_idx);
+    for (int b = 0; b < num_seqs; ++b) {
+        const int s0 = seq_start[b], L = seq_len[b];
+        // sequence b alone: its tokens are rows 0..L-1 of shifted tensors, and the top-k
+        // adds s0 to the selected positions so that they name packed rows
+        const __nv_bfloat16* qs = qb + (size_t)s0 * H_I * D_I;
+        const __nv_bfloat16* ks = kb + (size_t)s0 * D_I;
+        const float* ws = w + (size_t)s0 * H_I;
+        for (long long q0 = 0; q0 < L; q0 += rw) {
+            const int rows = (int)(L - q0 < rw ? L - q0 : rw);
+            cudaError_t e;
+            if (L > k) {  // otherwise every row selects all of its keys without reading scores
+                e = launch_indexer_bf16_prefill(qs, ks, ws, (int)q0 + rows, L, (int)q0, rows,
+                                                scores, ld, cs, ctx);
+                if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
+            }
+            e = launch_topk(scores, ld, rows, (int)q0, nullptr, L, k,
+                            idx + ((long long)s0 + q0) * ld_idx, ld_idx, cs, ctx, nullptr, s0);
+            if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
+        }
+    }
+    return DSA_OK;
+}
+
 size_t dsa_layer_stack_workspace_size(int T, int rows_window) {
     if (T <= 0) return 0;
     const long long ld = ((long long)T + 3) / 4 * 4;

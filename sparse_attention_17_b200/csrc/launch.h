@@ -63,10 +63,12 @@ cudaError_t launch_indexer_bf16_decode(const __nv_bfloat16* q_idx, const __nv_bf
                                        long long ld, cudaStream_t stream, const DevCtx& ctx);
 
 // Per-row top-k of dense score rows.  With row_mask non-null, only rows r with
-// row_mask[r] != 0 are processed (the filtered path's fallback).
+// row_mask[r] != 0 are processed (the filtered path's fallback).  idx_offset is added to
+// every selected key position (the first token of a packed sequence).
 cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin,
                         const int* row_len, int max_len, int k, int* idx, long long ld_idx,
-                        cudaStream_t stream, const DevCtx& ctx, const int* row_mask = nullptr);
+                        cudaStream_t stream, const DevCtx& ctx, const int* row_mask = nullptr,
+                        int idx_offset = 0);
 
 // Sampled keys per row the threshold kernel holds at most (tiles x 128).
 int topk_sample_max();

@@ -308,7 +308,8 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
 // Keeps the first `need` ties (tie bitmap) in index order, merges them into the selection
 // bitmap and writes the selected key positions in ascending order, then -1 up to k.
 __device__ void trim_ties_and_compact(TopkScratch& sh, uint32_t* sel, const uint32_t* tie,
-                                      int nwords, uint32_t need, int k, int* out) {
+                                      int nwords, uint32_t need, int k, int* out,
+                                      int idx_offset = 0) {
     const int wpt = (nwords + kThreads - 1) / kThreads;
     const int w0 = threadIdx.x * wpt;
     const int w1 = min(w0 + wpt, nwords);
@@ -341,7 +342,7 @@ __device__ void trim_ties_and_compact(TopkScratch& sh, uint32_t* sel, const uint
         while (bits) {
             const int b = __ffs(bits) - 1;
             bits &= bits - 1u;
-            if (pos < (uint32_t)k) out[pos] = w * 32 + b;
+            if (pos < (uint32_t)k) out[pos] = w * 32 + b + idx_offset;
             ++pos;
         }
     }
@@ -351,7 +352,8 @@ __device__ void trim_ties_and_compact(TopkScratch& sh, uint32_t* sel, const uint
 __global__ void __launch_bounds__(kThreads, 2)
 topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
                   const int* __restrict__ row_len, int max_len, int k, int* __restrict__ idx,
-                  long long ld_idx, const int* __restrict__ row_mask, unsigned* __restrict__ err) {
+                  long long ld_idx, const int* __restrict__ row_mask, int idx_offset,
+                  unsigned* __restrict__ err) {
     if (row_mask != nullptr && row_mask[blockIdx.x] == 0) return;  // row not asked for
     extern __shared__ __align__(16) unsigned char smem_raw[];
     TopkScratch& sh = *reinterpret_cast<TopkScratch*>(smem_raw);
@@ -373,7 +375,7 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
     }
     int* out = idx + (long long)r * ld_idx;
     if (n <= k) {  // every valid key is selected
-        for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
+        for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i + idx_offset : -1;
         return;
     }
     const float* row = scores + (long long)r * ld;
@@ -479,7 +481,7 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
     }
     __syncthreads();
 
-    trim_ties_and_compact(sh, sel, tie, nwords, need, k, out);
+    trim_ties_and_compact(sh, sel, tie, nwords, need, k, out, idx_offset);
 }
 
 
@@ -623,13 +625,15 @@ size_t topk_smem_bytes(int max_len) {
 
 cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin,
                         const int* row_len, int max_len, int k, int* idx, long long ld_idx,
-                        cudaStream_t stream, const DevCtx& ctx, const int* row_mask) {
+                        cudaStream_t stream, const DevCtx& ctx, const int* row_mask,
+                        int idx_offset) {
     const size_t smem = topk_smem_bytes(max_len);
     cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     topk_radix_kernel<<<rows, kThreads, smem, stream>>>(scores, ld, q_begin, row_len, max_len, k,
-                                                        idx, ld_idx, row_mask, ctx.err);
+                                                        idx, ld_idx, row_mask, idx_offset,
+                                                        ctx.err);
     count_launch(DSA_KERNEL_TOPK);
     return cudaGetLastError();
 }

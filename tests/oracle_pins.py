@@ -436,4 +436,29 @@ def pin_fp8_attention_masked_sdpa(mutant=0):
     np.testing.assert_allclose(od, op, rtol=1e-12, atol=1e-15)
     np.testing.assert_allclose(ld, lp, rtol=1e-12, atol=1e-15)
 
+
+def pin_varlen_packed_sequences(mutant=0):
+    """Packed batch of independent prompts: scores worked out per sequence with numpy
+    (einsum, ReLU, head weights) and a stable full sort per row, indices shifted to packed
+    rows; every selected row lies in [seq_start, t]; a gap left between sequences (left
+    padding) stays at the fill value."""
+    r = _rng(40)
+    starts, lens = [0, 9, 30, 33], [9, 20, 0, 14]
+    N, H_I, D_I, k = 50, 2, 4, 6
+    q = r.integers(-3, 4, (N, H_I, D_I)).astype(np.float32)
+    kk = r.integers(-3, 4, (N, D_I)).astype(np.float32)
+    w = r.integers(1, 3, (N, H_I)).astype(np.float32)
+    got = O.prefill_indices_varlen(q, kk, w, starts, lens, k, fill=-9, mutant=mutant)
+    want = np.full((N, k), -9, np.int32)
+    for s0, L in zip(starts, lens):
+        for t in range(s0, s0 + L):
+            keys = np.arange(s0, t + 1)
+            dots = np.einsum("jd,sd->js", q[t].astype(np.float64), kk[keys].astype(np.float64))
+            sc = (w[t].astype(np.float64)[:, None] * np.maximum(dots, 0)).sum(0)
+            order = np.argsort(-sc, kind="stable")[:k]
+            sel = np.sort(keys[order])
+            want[t] = np.r_[sel, -np.ones(k - len(sel), np.int32)]
+            assert np.all((got[t][got[t] >= 0] >= s0) & (got[t][got[t] >= 0] <= t))
+    assert np.array_equal(got, want)
+
 ALL_PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

@@ -157,6 +157,27 @@ def test_fp8_attention_and_quantize_reject(lib):
     assert q(16, 8, 0.0, 16, None) == _lib.DSA_ERR_INVALID_ARG
 
 
+def test_index_varlen_rejects(lib):
+    f = lib.dsa_index_varlen
+    arr = ctypes.c_int * 3
+
+    def call(starts, lens, n=100, k=8, ld=8, ws_bytes=1 << 20, H_I=16):
+        return f(16, 16, 16, H_I, 64, n, len(starts), ctypes.cast(arr(*starts), ctypes.c_void_p),
+                 ctypes.cast(arr(*lens), ctypes.c_void_p), k, 16, ld, 16, ws_bytes, None)
+
+    assert call([0, 10], [20, 5]) == _lib.DSA_ERR_INVALID_ARG    # overlap
+    assert call([0, 90], [20, 20]) == _lib.DSA_ERR_INVALID_ARG   # past num_tokens
+    assert call([5, 0], [2, 2]) == _lib.DSA_ERR_INVALID_ARG      # not increasing
+    assert call([0], [-1]) == _lib.DSA_ERR_INVALID_ARG           # negative length
+    assert call([0], [10], k=0) == _lib.DSA_ERR_UNSUPPORTED
+    assert call([0], [10], ld=4) == _lib.DSA_ERR_INVALID_ARG     # ld_idx < k
+    assert call([0], [10], H_I=2) == _lib.DSA_ERR_UNSUPPORTED
+    assert call([0], [10], ws_bytes=16) == _lib.DSA_ERR_WORKSPACE
+    assert call([0, 3], [0, 0]) == _lib.DSA_OK                   # nothing to do
+    assert lib.dsa_index_varlen_workspace_size(100, 7) == 7 * 100 * 4
+    assert lib.dsa_index_varlen_workspace_size(65536, 0) == 4096 << 20
+
+
 def test_workspace_sizes(lib):
     assert lib.dsa_sparse_mla_workspace_size(0, 100, 16, 512, 2048) == 0
     ws = lib.dsa_sparse_mla_workspace_size(1, 64, 16, 512, 2048)

@@ -1,6 +1,6 @@
 """Mutation check of the pins: each deliberate mistake compiled into the oracle
 (ORACLE_MUTANT in dsa_oracle.c) must make at least one pin fail.  The mistakes are
-planted only in CPU builds of the oracle (mutants 9..12 in the oracle's Python fp8
+planted only in CPU builds of the oracle (mutants 9..13 in the oracle's Python
 functions)."""
 import pytest
 
@@ -20,6 +20,7 @@ MUTANTS = {
     10: "E4M3 subnormals decoded as normals",
     11: "E4M3 encoder ties away from zero",
     12: "fp8 attention output without kv_scale",
+    13: "varlen indices without the packed offset",
 }
 
 
