@@ -338,6 +338,17 @@ size_t dsa_layer_stack_workspace_size(int T, int rows_window);
  */
 dsa_status dsa_pattern_from_freq(int freq, int num_layers, char* out, int out_len);
 
+/*
+ * dsa_selftest_wait_timeout -- runs the failure path of the kernels' pipeline waits: one
+ * CTA waits on an mbarrier that nothing arrives on, with the same time-bounded wait every
+ * kernel uses (2 s).  The wait gives up, records DSA_DEVERR_TIMEOUT in the device error
+ * word (read it with dsa_check_device_errors) and the kernel exits; *gave_up (a device
+ * int) receives 1.  No memory other than the error word and *gave_up is touched, and the
+ * context stays usable.  Not part of the hot path: a check that a hung pipeline stage
+ * becomes an error status instead of a hung GPU.
+ */
+dsa_status dsa_selftest_wait_timeout(int* gave_up, dsa_stream_t stream);
+
 /* Reads and clears the current device's error word after synchronizing `stream`.
  * *error_bits (may be NULL) receives the DSA_DEVERR_* bits.  Returns
  * DSA_ERR_DEVICE_CHECK if any bit was set, DSA_OK otherwise. */

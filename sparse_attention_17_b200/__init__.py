@@ -6,5 +6,6 @@ from ._lib import (KERNEL_KINDS, DSAError, check_device_errors, index_select,  #
                    index_select_workspace_size, index_varlen,
                    index_varlen_workspace_size, indexer_scores, latent_quantize_fp8,
                    launch_count, layer_stack, layer_stack_workspace_size, lib_path, load,
-                   pattern_from_freq, reset_launch_counts, sparse_mla_fp8_fwd, sparse_mla_fwd,
+                   pattern_from_freq, reset_launch_counts, selftest_wait_timeout,
+                   sparse_mla_fp8_fwd, sparse_mla_fwd,
                    sparse_mla_workspace_size, topk_select)

@@ -49,6 +49,7 @@ SYMBOLS = [
                              _P, _P, _P, _P, _P, _SZ, _P]),
     ("dsa_layer_stack_workspace_size", _SZ, [_I, _I]),
     ("dsa_pattern_from_freq", _I, [_I, _I, ctypes.c_char_p, _I]),
+    ("dsa_selftest_wait_timeout", _I, [_P, _P]),
     ("dsa_check_device_errors", _I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     ("dsa_launch_count", _LL, [_I]),
     ("dsa_reset_launch_counts", None, []),
@@ -303,6 +304,12 @@ def index_varlen(q_idx, k_idx, w, seq_start, seq_len, k: int, idx, workspace) ->
                                 ctypes.cast(lens, ctypes.c_void_p), k, idx.data_ptr(),
                                 idx.stride(0), workspace.data_ptr(),
                                 workspace.numel() * workspace.element_size(), _stream()))
+
+
+def selftest_wait_timeout(gave_up) -> None:
+    """dsa_selftest_wait_timeout: gave_up is a 1-element int32 CUDA tensor."""
+    _need(gave_up, torch.int32, 1, "gave_up")
+    _check(load().dsa_selftest_wait_timeout(gave_up.data_ptr(), _stream()))
 
 
 def latent_quantize_fp8(src, kv_scale: float, dst) -> None:

@@ -447,6 +447,16 @@ dsa_status dsa_index_varlen(const void* q_idx, const void* k_idx, const float* w
     return DSA_OK;
 }
 
+dsa_status dsa_selftest_wait_timeout(int* gave_up, dsa_stream_t stream) {
+    g_last_error[0] = 0;
+    if (!gave_up || !aligned16(gave_up)) return fail(DSA_ERR_INVALID_ARG, "gave_up must be a 16-byte aligned device int");
+    DevCtx ctx;
+    dsa_status st = check_stream_device(&ctx);
+    if (st != DSA_OK) return st;
+    cudaError_t e = launch_wait_timeout_selftest(gave_up, reinterpret_cast<cudaStream_t>(stream), ctx);
+    return e == cudaSuccess ? DSA_OK : cuda_fail(e, "self-test launch");
+}
+
 size_t dsa_layer_stack_workspace_size(int T, int rows_window) {
     if (T <= 0) return 0;
     const long long ld = ((long long)T + 3) / 4 * 4;

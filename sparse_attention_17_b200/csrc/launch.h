@@ -111,6 +111,9 @@ cudaError_t launch_sparse_mla_mma(const __nv_bfloat16* q, const void* kv, bool k
 cudaError_t launch_latent_quantize_fp8(const __nv_bfloat16* src, long long n, float kv_scale,
                                        uint8_t* dst, cudaStream_t stream, const DevCtx& ctx);
 
+// One CTA whose bounded mbarrier wait runs out (2 s); *gave_up <- 1 if it gave up.
+cudaError_t launch_wait_timeout_selftest(int* gave_up, cudaStream_t stream, const DevCtx& ctx);
+
 cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int num_q, int splits,
                                __nv_bfloat16* out, float* lse, cudaStream_t stream);
 

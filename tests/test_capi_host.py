@@ -178,6 +178,11 @@ def test_index_varlen_rejects(lib):
     assert lib.dsa_index_varlen_workspace_size(65536, 0) == 4096 << 20
 
 
+def test_selftest_rejects_bad_pointer(lib):
+    assert lib.dsa_selftest_wait_timeout(None, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_selftest_wait_timeout(18, None) == _lib.DSA_ERR_INVALID_ARG
+
+
 def test_workspace_sizes(lib):
     assert lib.dsa_sparse_mla_workspace_size(0, 100, 16, 512, 2048) == 0
     ws = lib.dsa_sparse_mla_workspace_size(1, 64, 16, 512, 2048)
