@@ -54,6 +54,7 @@ struct IdxSmem {
     uint64_t acc_full[2], acc_empty[2];
     uint32_t tmem_base;
     int abort;
+    int pages[kDecodeChunkTiles * kBM / 16];  // decode: the unit's page-table entries
 };
 
 // What the prefill epilogue does with each score.
@@ -156,6 +157,44 @@ __device__ __forceinline__ UnitInfo<QB, PAGED> unit_info(const IdxParams& p, int
     return x;
 }
 
+// One unit's copies, issued by the producer thread: the query block and its head weights
+// (once the previous user of the buffer is done), then every key tile into the ring.
+// Paged keys read their pool rows from sm.pages (filled by the producer warp).  Returns
+// false when a wait gave up.
+template <int QB, bool PAGED>
+__device__ __forceinline__ bool produce_unit(IdxSmem<QB>& sm, const IdxParams& p,
+                                             const UnitInfo<QB, PAGED>& x, int ui, uint32_t& it,
+                                             const CUtensorMap* tmap_q, const CUtensorMap* tmap_k,
+                                             volatile int* abort) {
+    const int qb = ui & 1;
+    if (!mbar_wait(&sm.q_empty[qb], ((ui >> 1) & 1) ^ 1, abort, p.err)) return false;
+    // query block (TMA, swizzled) and its head weights (bulk copy) on one barrier
+    const int nq = PAGED ? 1 : x.len;
+    const uint32_t wbytes = (uint32_t)nq * kHI * 4;
+    mbar_arrive_expect_tx(&sm.q_full[qb], (uint32_t)(QB * kHI * 128) + wbytes);
+    tma_load_2d(sm.q[qb], tmap_q, 0, x.row0 * kHI, &sm.q_full[qb]);
+    bulk_load(sm.w[qb], p.w + (long long)x.row0 * kHI, wbytes, &sm.q_full[qb]);
+    for (int j = 0; j < x.ntiles; ++j, ++it) {
+        const int st = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (!mbar_wait(&sm.k_empty[st], ph ^ 1, abort, p.err)) return false;
+        const int tile = (x.tile0 + j) * (PAGED ? 1 : p.tile_stride);
+        if constexpr (!PAGED) {
+            mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
+            tma_load_2d(sm.k[st], tmap_k, 0, tile * kBM, &sm.k_full[st]);
+        } else {
+            const int ps = p.page_size;
+            const int per = kBM / ps;
+            const int used = min(per, (x.len - tile * kBM + ps - 1) / ps);
+            mbar_arrive_expect_tx(&sm.k_full[st], (uint32_t)(used * ps * 128));
+            for (int q = 0; q < used; ++q)
+                tma_load_2d(sm.k[st] + q * ps * 128, tmap_k, 0, sm.pages[j * per + q] * ps,
+                            &sm.k_full[st]);
+        }
+    }
+    return true;
+}
+
 template <int QB, bool PAGED, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
@@ -200,48 +239,38 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0 && lane == 0) {
+    if (warp == 0) {
         // ---------------- TMA producer ----------------
-        tma_prefetch_desc(&tmap_q);
-        tma_prefetch_desc(&tmap_k);
+        // Lane 0 issues the copies.  For paged keys the whole warp first reads the unit's
+        // page-table entries into shared memory: one round trip per unit instead of a
+        // dependent load before every tile's copies.
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_q);
+            tma_prefetch_desc(&tmap_k);
+        }
         uint32_t it = 0;
         for (int i = 0, ui = 0;; ++i, ++ui) {
             const int u = unit_at(i);
             if (u >= p.num_units) break;
             const UnitInfo<QB, PAGED> x = unit_info<QB, PAGED>(p, u);
-            const int qb = ui & 1;
-            if (!mbar_wait(&sm.q_empty[qb], ((ui >> 1) & 1) ^ 1, abort, p.err)) break;
-            // query block (TMA, swizzled) and its head weights (bulk copy) on one barrier
-            const int nq = PAGED ? 1 : x.len;
-            const uint32_t wbytes = (uint32_t)nq * kHI * 4;
-            mbar_arrive_expect_tx(&sm.q_full[qb], kQBytes + wbytes);
-            tma_load_2d(sm.q[qb], &tmap_q, 0, x.row0 * kHI, &sm.q_full[qb]);
-            bulk_load(sm.w[qb], p.w + (long long)x.row0 * kHI, wbytes, &sm.q_full[qb]);
-            bool ok = true;
-            for (int j = 0; j < x.ntiles; ++j, ++it) {
-                const int st = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
-                if (!mbar_wait(&sm.k_empty[st], ph ^ 1, abort, p.err)) { ok = false; break; }
-                const int tile = (x.tile0 + j) * (PAGED ? 1 : p.tile_stride);
-                if constexpr (!PAGED) {
-                    mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
-                    tma_load_2d(sm.k[st], &tmap_k, 0, tile * kBM, &sm.k_full[st]);
-                } else {
-                    const int ps = p.page_size;
-                    const int per = kBM / ps;
-                    const int page0 = tile * per;
-                    const int used = min(per, (x.len - tile * kBM + ps - 1) / ps);
-                    mbar_arrive_expect_tx(&sm.k_full[st], (uint32_t)(used * ps * 128));
-                    for (int q = 0; q < used; ++q) {
-                        int pg = __ldg(p.page_table + (long long)x.row0 * p.max_pages + page0 + q);
-                        if (pg < 0 || pg >= p.num_pages) {
-                            atomicOr(p.err, DSA_DEVERR_PAGE_RANGE);
-                            pg = 0;
-                        }
-                        tma_load_2d(sm.k[st] + q * ps * 128, &tmap_k, 0, pg * ps, &sm.k_full[st]);
+            if constexpr (PAGED) {
+                const int per = kBM / p.page_size;
+                const int npg = min(x.ntiles * per, (x.len - x.tile0 * kBM + p.page_size - 1) / p.page_size);
+                const int* pt = p.page_table + (long long)x.row0 * p.max_pages + x.tile0 * per;
+                for (int q = lane; q < npg; q += 32) {
+                    int pg = __ldg(pt + q);
+                    if (pg < 0 || pg >= p.num_pages) {
+                        atomicOr(p.err, DSA_DEVERR_PAGE_RANGE);
+                        pg = 0;
                     }
+                    sm.pages[q] = pg;
                 }
+                __syncwarp();
             }
+            bool ok = true;
+            if (lane == 0) ok = produce_unit<QB, PAGED>(sm, p, x, ui, it, &tmap_q, &tmap_k, abort);
+            ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+            __syncwarp();  // lane 0 has issued every copy that reads sm.pages
             if (!ok) break;
         }
     } else if (warp == 1 && lane == 0) {
