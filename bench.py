@@ -361,10 +361,37 @@ def run_native(args, rank, world, local_rank):
         torch.cuda.synchronize()
         e2e_ms = s2.elapsed_time(t2) / n_e2e
         e2e_ms = max_over_ranks(e2e_ms, dev)
+
+        # the copies alone, each direction on its own stream: the host link's bound on e2e
+        def copy_ms(fn, st, reps=3):
+            fn()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            for _ in range(reps):
+                fn()
+            b.record(st)
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / reps
+
+        def up():
+            with torch.cuda.stream(s_up):
+                for nme in names:
+                    xs[1][nme].copy_(pinned[nme], non_blocking=True)
+
+        def down():
+            with torch.cuda.stream(s_down):
+                out_host[1].copy_(outs[1], non_blocking=True)
+
+        h2d_ms = copy_ms(up, s_up)
+        d2h_ms = copy_ms(down, s_down)
         e2e = {"value": aggregate_tokens_per_s(T, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "steps": n_e2e, "overlap": "double-buffered inputs/outputs, copies on their own streams"}
+               "steps": n_e2e, "overlap": "double-buffered inputs/outputs, copies on their own streams",
+               "h2d_gbs_alone": round(h2d / (h2d_ms / 1e3) / 1e9, 1),
+               "d2h_gbs_alone": round(d2h / (d2h_ms / 1e3) / 1e9, 1),
+               "copy_bound_ms": round(max(h2d_ms, d2h_ms), 3)}
 
     result = None
     if rank == 0:
@@ -489,6 +516,17 @@ def run_decode(args, local_rank):
     t_idx = _timed(indexer, args.steps, 1, stream)
     t_topk = _timed(topk, args.steps, 1, stream)
     t_mla = _timed(mla, args.steps, 1, stream)
+    # the same step captured once as a CUDA graph (serving stacks replay decode steps so)
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        step()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    ms_graph = _timed(graph.replay, args.steps, args.warmup, stream)
     assert dsa.check_device_errors() == 0
     peaks, src = load_peaks()
     gather = B * k * (576 if fp8 else 1152)
@@ -501,6 +539,8 @@ def run_decode(args, local_rank):
                        "page_size": 64, "kv_cache": "e4m3 x kv_scale" if fp8 else "bf16"},
             "kernels": {"indexer_ms": round(t_idx, 4), "topk_ms": round(t_topk, 4),
                         "sparse_mla_decode_ms": round(t_mla, 4)},
+            "cuda_graph": {"ms_per_step": round(ms_graph, 4),
+                           "value": round(B / (ms_graph / 1e3), 1)},
             "derived": {"indexer_key_read_gbs": round(kidx / (t_idx / 1e3) / 1e9, 1),
                         "mla_gather_gbs": round(gather / (t_mla / 1e3) / 1e9, 1),
                         "mla_gather_frac_of_hbm": round(gather / (t_mla / 1e3) / 1e9
