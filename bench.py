@@ -385,13 +385,35 @@ def run_native(args, rank, world, local_rank):
 
         h2d_ms = copy_ms(up, s_up)
         d2h_ms = copy_ms(down, s_down)
+
+        def both():  # one step's upload and download at the same time, as in the pipeline
+            up()
+            down()
+
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        stream.synchronize()
+        a.record(stream)
+        s_up.wait_event(a)
+        s_down.wait_event(a)
+        for _ in range(3):
+            both()
+        ev_u, ev_d = torch.cuda.Event(), torch.cuda.Event()
+        ev_u.record(s_up)
+        ev_d.record(s_down)
+        stream.wait_event(ev_u)
+        stream.wait_event(ev_d)
+        b.record(stream)
+        torch.cuda.synchronize()
+        both_ms = a.elapsed_time(b) / 3
         e2e = {"value": aggregate_tokens_per_s(T, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "steps": n_e2e, "overlap": "double-buffered inputs/outputs, copies on their own streams",
                "h2d_gbs_alone": round(h2d / (h2d_ms / 1e3) / 1e9, 1),
                "d2h_gbs_alone": round(d2h / (d2h_ms / 1e3) / 1e9, 1),
-               "copy_bound_ms": round(max(h2d_ms, d2h_ms), 3)}
+               "copy_bound_ms": round(max(h2d_ms, d2h_ms), 3),
+               "copy_both_directions_ms": round(both_ms, 3)}
 
     result = None
     if rank == 0:
