@@ -200,7 +200,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                   const __grid_constant__ CUtensorMap tmap_k, const IdxParams p) {
     constexpr int BN = QB * kHI;                     // UMMA N
-    constexpr uint32_t kQBytes = BN * 128;
     constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;  // TMEM columns per accumulator
     constexpr uint32_t kTmemCols = 2 * kAccCols <= 32 ? 32 : (2 * kAccCols <= 64 ? 64 : (2 * kAccCols <= 128 ? 128 : (2 * kAccCols <= 256 ? 256 : 512)));
     constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, 0, 0);

@@ -106,7 +106,7 @@ struct MmaSmem {
     alignas(128) uint8_t p[L::kStages][kPBytes];
     alignas(16) int valid[L::kStages][kBK];  // 1: the staged row holds the key; -1: not fetched
     alignas(16) float spart[kComputeWarps][kNT][32][4];  // [from warp][n-tile] partial scores
-    alignas(16) float red[L::kStages][kComputeWarps][kH];  // per warp, per head block maxima
+    alignas(16) float red[L::kStages][kH][kComputeWarps];  // per head, per warp block maxima
     alignas(16) float lsum[2][kComputeWarps][kH];         // per warp row sums at the end of a unit
     uint64_t a_full[L::kStages], a_free[L::kStages];
     uint64_t q_full, q_empty;
@@ -441,16 +441,16 @@ sparse_mla_mma_kernel(const Params p) {
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
                 if (t == 0) {
-                    sm.red[s][warp][g] = mx0;
-                    sm.red[s][warp][g + 8] = mx1;
+                    sm.red[s][g][warp] = mx0;
+                    sm.red[s][g + 8][warp] = mx1;
                 }
                 compute_sync();
                 float ref[2], alpha[2];
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
-                    float bm = sm.red[s][0][g + 8 * r];
-#pragma unroll
-                    for (int i = 1; i < kComputeWarps; ++i) bm = fmaxf(bm, sm.red[s][i][g + 8 * r]);
+                    static_assert(kComputeWarps == 4, "one 16-byte load of the warps' maxima");
+                    const float4 wm = *reinterpret_cast<const float4*>(sm.red[s][g + 8 * r]);
+                    const float bm = fmaxf(fmaxf(wm.x, wm.y), fmaxf(wm.z, wm.w));
                     const float mn = fmaxf(m_run[r], bm);
                     alpha[r] = m_run[r] == -INFINITY ? 0.f : exp2f(m_run[r] - mn);
                     m_run[r] = mn;
