@@ -5,9 +5,10 @@
 // n <= k every key is selected.  Output: the selected key positions in ascending order,
 // then -1 padding.
 //
-// One CTA of 512 threads per row.  Scores map to order-preserving uint32 keys.  Each warp
-// owns a 512-entry slice of the shared candidate buffer, so candidates are appended with
-// a ballot and a popcount and no shared atomics.
+// One CTA per row: 512 threads, or 1024 when the launch has fewer rows than the GPU has
+// SMs (a decode batch).  Scores map to order-preserving uint32 keys.  Each warp owns a
+// slice of the shared candidate buffer (512 entries, or 256 with 1024 threads), so
+// candidates are appended with a ballot and a popcount and no shared atomics.
 // Fast path (one read of the row):
 //   sample  every 16th 32-key chunk of the row (at most 256 chunks, all loads in flight
 //           at once) goes to the slices; a two-round (12 + 12 bit) radix select there
@@ -29,30 +30,37 @@ namespace dsa {
 
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 4096;
 constexpr int kCandCap = 8192;
-constexpr int kStride = kWarps * 32;  // elements covered by all warps per iteration
-constexpr int kSlice = kCandCap / kWarps;  // candidate entries owned by one warp
 constexpr int kUnroll = 4;                 // 16-byte loads in flight per thread
 constexpr int kBM_SAMPLE = 128;            // keys per sampled tile (the indexer's tile)
+constexpr int kMaxWarps = 32;
+constexpr int kSampleChunks = kCandCap / 32;  // at most 256 sampled 32-key chunks
+
+// The block size: 512 threads (two CTAs per SM) when rows are plentiful, 1024 (one CTA
+// per SM) for launches with fewer rows than SMs, such as a decode batch.
+template <int T>
+struct TopkCfg {
+    static constexpr int kThreads = T;
+    static constexpr int kWarps = T / 32;
+    static constexpr int kStride = kWarps * 32;          // elements covered per iteration
+    static constexpr int kSlice = kCandCap / kWarps;     // candidate entries of one warp
+    static constexpr int kSampleChunksPerWarp = kSampleChunks / kWarps;  // one slice
+    // rows this short make every key a candidate: each warp's 128-key chunks fit its slice
+    static constexpr int kNoSampleMax = (kSlice / 128) * 128 * kWarps;
+    static_assert(kWarps <= kMaxWarps && kSlice % 128 == 0, "block size");
+};
 
 struct TopkScratch {
     uint32_t hist[kBins];
     uint32_t cand_key[kCandCap];
     int cand_idx[kCandCap];
-    uint32_t scan[kWarps];
-    uint32_t wcount[kWarps];  // candidates appended by each warp (may exceed kSlice)
+    uint32_t scan[kMaxWarps];
+    uint32_t wcount[kMaxWarps];  // candidates appended by each warp (may exceed its slice)
     uint32_t cand_count;
     uint32_t found_bin;
     uint32_t found_above;
 };
-
-constexpr int kSampleChunks = kCandCap / 32;  // at most 256 sampled 32-key chunks
-constexpr int kSampleChunksPerWarp = kSampleChunks / kWarps;  // 16 chunks = one slice
-// rows this short make every key a candidate: each warp's 128-key chunks fit its slice
-constexpr int kNoSampleMax = (kSlice / 128) * 128 * kWarps;
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
@@ -70,6 +78,7 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool pred
 }
 
 // Exclusive prefix sum over the block's threads (in thread order); *total gets the sum.
+template <int T>
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, TopkScratch& sh,
                                                          uint32_t* total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -82,31 +91,32 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, TopkScratch
     if (lane == 31) sh.scan[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        uint32_t w = lane < kWarps ? sh.scan[lane] : 0u;
+        uint32_t w = lane < TopkCfg<T>::kWarps ? sh.scan[lane] : 0u;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
             if (lane >= o) w += y;
         }
-        if (lane < kWarps) sh.scan[lane] = w;
+        if (lane < TopkCfg<T>::kWarps) sh.scan[lane] = w;
     }
     __syncthreads();
     const uint32_t before = (warp > 0 ? sh.scan[warp - 1] : 0u) + x - v;
-    *total = sh.scan[kWarps - 1];
+    *total = sh.scan[TopkCfg<T>::kWarps - 1];
     __syncthreads();
     return before;
 }
 
 // Finds the bin b (scanning from the top) with above(b) < need <= above(b) + hist[b],
 // above(b) = number of keys in bins higher than b.  Result in sh.found_bin/found_above.
+template <int T>
 __device__ void find_bin(TopkScratch& sh, int nbins, uint32_t need) {
-    const int per = nbins >= kThreads ? nbins / kThreads : 1;
+    const int per = nbins >= TopkCfg<T>::kThreads ? nbins / TopkCfg<T>::kThreads : 1;
     const int first = nbins - 1 - (int)threadIdx.x * per;  // this thread's highest bin
     uint32_t local = 0;
     if (first >= 0)
         for (int i = 0; i < per; ++i) local += sh.hist[first - i];
     uint32_t total;
-    uint32_t above = block_exclusive_scan(local, sh, &total);
+    uint32_t above = block_exclusive_scan<T>(local, sh, &total);
     if (first >= 0 && above < need && above + local >= need) {
         for (int i = 0; i < per; ++i) {
             const uint32_t c = sh.hist[first - i];
@@ -121,31 +131,33 @@ __device__ void find_bin(TopkScratch& sh, int nbins, uint32_t need) {
     __syncthreads();
 }
 
+template <int T>
 __device__ __forceinline__ void zero_hist(TopkScratch& sh, int nbins) {
-    for (int i = threadIdx.x; i < nbins; i += kThreads) sh.hist[i] = 0u;
+    for (int i = threadIdx.x; i < nbins; i += TopkCfg<T>::kThreads) sh.hist[i] = 0u;
 }
 
-// Radix select over the warps' candidate slices (warp w owns cand_key[w * kSlice ..] with
-// wcount[w] <= kSlice entries).  exact: returns the need-th largest key tau and sets
+// Radix select over the warps' candidate slices (warp w owns cand_key[w * TopkCfg<T>::kSlice ..] with
+// wcount[w] <= TopkCfg<T>::kSlice entries).  exact: returns the need-th largest key tau and sets
 // *need_out to how many keys equal to tau belong to the top `need` (12 + 12 + 8 bits).
 // !exact: stops after 24 bits and returns the lower edge of the 24-bit bin holding the
 // need-th largest key, a lower bound of it.
+template <int T>
 __device__ uint32_t slice_radix_select(TopkScratch& sh, uint32_t need, bool exact,
                                        uint32_t* need_out) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t* keys = sh.cand_key + warp * kSlice;
+    const uint32_t* keys = sh.cand_key + warp * TopkCfg<T>::kSlice;
     const int cnt = (int)sh.wcount[warp];
-    zero_hist(sh, kBins);
+    zero_hist<T>(sh, kBins);
     __syncthreads();
     for (int c0 = 0; c0 < cnt; c0 += 32) {
         const int c = c0 + lane;
         hist_add(sh.hist, c < cnt ? keys[c] >> 20 : 0u, c < cnt);
     }
     __syncthreads();
-    find_bin(sh, kBins, need);
+    find_bin<T>(sh, kBins, need);
     const uint32_t b1 = sh.found_bin;
     need -= sh.found_above;
-    zero_hist(sh, kBins);
+    zero_hist<T>(sh, kBins);
     __syncthreads();
     for (int c0 = 0; c0 < cnt; c0 += 32) {
         const int c = c0 + lane;
@@ -153,7 +165,7 @@ __device__ uint32_t slice_radix_select(TopkScratch& sh, uint32_t need, bool exac
         hist_add(sh.hist, (key >> 8) & 0xFFFu, c < cnt && (key >> 20) == b1);
     }
     __syncthreads();
-    find_bin(sh, kBins, need);
+    find_bin<T>(sh, kBins, need);
     const uint32_t pre = (b1 << 12) | sh.found_bin;
     need -= sh.found_above;
     if (!exact) {
@@ -161,7 +173,7 @@ __device__ uint32_t slice_radix_select(TopkScratch& sh, uint32_t need, bool exac
         __syncthreads();
         return pre << 8;
     }
-    zero_hist(sh, 256);
+    zero_hist<T>(sh, 256);
     __syncthreads();
     for (int c0 = 0; c0 < cnt; c0 += 32) {
         const int c = c0 + lane;
@@ -169,7 +181,7 @@ __device__ uint32_t slice_radix_select(TopkScratch& sh, uint32_t need, bool exac
         hist_add(sh.hist, key & 0xFFu, c < cnt && (key >> 8) == pre);
     }
     __syncthreads();
-    find_bin(sh, 256, need);
+    find_bin<T>(sh, 256, need);
     need -= sh.found_above;
     *need_out = need;
     const uint32_t tau = (pre << 8) | sh.found_bin;
@@ -180,19 +192,20 @@ __device__ uint32_t slice_radix_select(TopkScratch& sh, uint32_t need, bool exac
 // Exact selection from global memory (fallback): histogram passes over the whole row.
 // Fills sel (keys above the k-th largest) and tie (keys equal to it); returns how many
 // of the ties belong to the top k.  sel must be zero, tie zero on entry.
+template <int T>
 __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ row, int n,
                                      int k, uint32_t* sel, uint32_t* tie) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // ---- pass 1: histogram of the top 12 key bits over the whole row ----
-    zero_hist(sh, kBins);
+    zero_hist<T>(sh, kBins);
     if (threadIdx.x == 0) sh.cand_count = 0u;
     __syncthreads();
-    for (int base = warp * 32; base < n; base += 4 * kStride) {
+    for (int base = warp * 32; base < n; base += 4 * TopkCfg<T>::kStride) {
         float x[4];
         bool in[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const int s = base + u * kStride + lane;
+            const int s = base + u * TopkCfg<T>::kStride + lane;
             in[u] = s < n;
             x[u] = in[u] ? __ldg(row + s) : 0.f;
         }
@@ -200,7 +213,7 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
         for (int u = 0; u < 4; ++u) hist_add(sh.hist, float_order_key(x[u]) >> 20, in[u]);
     }
     __syncthreads();
-    find_bin(sh, kBins, (uint32_t)k);
+    find_bin<T>(sh, kBins, (uint32_t)k);
     const uint32_t b1 = sh.found_bin;
     uint32_t need = (uint32_t)k - sh.found_above;
     const uint32_t cnt1 = sh.hist[b1];
@@ -209,7 +222,7 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
     uint32_t tau;
     if (cnt1 <= (uint32_t)kCandCap) {
         // ---- pass 2: definite selections to the bitmap, the b1 bucket to shared memory ----
-        for (int base = warp * 32; base < n; base += kStride) {
+        for (int base = warp * 32; base < n; base += TopkCfg<T>::kStride) {
             const int s = base + lane;
             const bool in = s < n;
             const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
@@ -229,34 +242,34 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
                 }
             }
         }
-        zero_hist(sh, kBins);
+        zero_hist<T>(sh, kBins);
         __syncthreads();
         const int cnt = (int)sh.cand_count;
         // ---- refine: bits 19..8 ----
-        for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
+        for (int c0 = warp * 32; c0 < cnt; c0 += TopkCfg<T>::kStride) {
             const int c = c0 + lane;
             const bool in = c < cnt;
             hist_add(sh.hist, in ? (sh.cand_key[c] >> 8) & 0xFFFu : 0u, in);
         }
         __syncthreads();
-        find_bin(sh, kBins, need);
+        find_bin<T>(sh, kBins, need);
         const uint32_t b2 = sh.found_bin;
         need -= sh.found_above;
-        zero_hist(sh, 256);
+        zero_hist<T>(sh, 256);
         __syncthreads();
         // ---- refine: bits 7..0 ----
         const uint32_t pre = (b1 << 12) | b2;
-        for (int c0 = warp * 32; c0 < cnt; c0 += kStride) {
+        for (int c0 = warp * 32; c0 < cnt; c0 += TopkCfg<T>::kStride) {
             const int c = c0 + lane;
             const uint32_t key = c < cnt ? sh.cand_key[c] : 0u;
             const bool in = c < cnt && (key >> 8) == pre;
             hist_add(sh.hist, key & 0xFFu, in);
         }
         __syncthreads();
-        find_bin(sh, 256, need);
+        find_bin<T>(sh, 256, need);
         need -= sh.found_above;
         tau = (pre << 8) | sh.found_bin;
-        for (int c = threadIdx.x; c < cnt; c += kThreads) {
+        for (int c = threadIdx.x; c < cnt; c += TopkCfg<T>::kThreads) {
             const uint32_t key = sh.cand_key[c];
             const int s = sh.cand_idx[c];
             if (key > tau) atomicOr(&sel[s >> 5], 1u << (s & 31));
@@ -264,32 +277,32 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
         }
     } else {
         // ---- the b1 bucket does not fit: refine from global memory ----
-        zero_hist(sh, kBins);
+        zero_hist<T>(sh, kBins);
         __syncthreads();
-        for (int base = warp * 32; base < n; base += kStride) {
+        for (int base = warp * 32; base < n; base += TopkCfg<T>::kStride) {
             const int s = base + lane;
             const bool in = s < n;
             const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
             hist_add(sh.hist, (key >> 8) & 0xFFFu, in && (key >> 20) == b1);
         }
         __syncthreads();
-        find_bin(sh, kBins, need);
+        find_bin<T>(sh, kBins, need);
         const uint32_t b2 = sh.found_bin;
         need -= sh.found_above;
-        zero_hist(sh, 256);
+        zero_hist<T>(sh, 256);
         __syncthreads();
         const uint32_t pre = (b1 << 12) | b2;
-        for (int base = warp * 32; base < n; base += kStride) {
+        for (int base = warp * 32; base < n; base += TopkCfg<T>::kStride) {
             const int s = base + lane;
             const bool in = s < n;
             const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
             hist_add(sh.hist, key & 0xFFu, in && (key >> 8) == pre);
         }
         __syncthreads();
-        find_bin(sh, 256, need);
+        find_bin<T>(sh, 256, need);
         need -= sh.found_above;
         tau = (pre << 8) | sh.found_bin;
-        for (int base = warp * 32; base < n; base += kStride) {
+        for (int base = warp * 32; base < n; base += TopkCfg<T>::kStride) {
             const int s = base + lane;
             const bool in = s < n;
             const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
@@ -307,16 +320,17 @@ __device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ 
 
 // Keeps the first `need` ties (tie bitmap) in index order, merges them into the selection
 // bitmap and writes the selected key positions in ascending order, then -1 up to k.
+template <int T>
 __device__ void trim_ties_and_compact(TopkScratch& sh, uint32_t* sel, const uint32_t* tie,
                                       int nwords, uint32_t need, int k, int* out,
                                       int idx_offset = 0) {
-    const int wpt = (nwords + kThreads - 1) / kThreads;
+    const int wpt = (nwords + TopkCfg<T>::kThreads - 1) / TopkCfg<T>::kThreads;
     const int w0 = threadIdx.x * wpt;
     const int w1 = min(w0 + wpt, nwords);
     uint32_t local = 0;
     for (int w = w0; w < w1; ++w) local += __popc(tie[w]);
     uint32_t total;
-    uint32_t before = block_exclusive_scan(local, sh, &total);
+    uint32_t before = block_exclusive_scan<T>(local, sh, &total);
     for (int w = w0; w < w1; ++w) {
         uint32_t tb = tie[w];
         const uint32_t c = __popc(tb);
@@ -336,7 +350,7 @@ __device__ void trim_ties_and_compact(TopkScratch& sh, uint32_t* sel, const uint
     __syncthreads();
     local = 0;
     for (int w = w0; w < w1; ++w) local += __popc(sel[w]);
-    uint32_t pos = block_exclusive_scan(local, sh, &total);
+    uint32_t pos = block_exclusive_scan<T>(local, sh, &total);
     for (int w = w0; w < w1; ++w) {
         uint32_t bits = sel[w];
         while (bits) {
@@ -346,10 +360,11 @@ __device__ void trim_ties_and_compact(TopkScratch& sh, uint32_t* sel, const uint
             ++pos;
         }
     }
-    for (int i = (int)total + threadIdx.x; i < k; i += kThreads) out[i] = -1;
+    for (int i = (int)total + threadIdx.x; i < k; i += TopkCfg<T>::kThreads) out[i] = -1;
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+template <int T>
+__global__ void __launch_bounds__(T, T <= 512 ? 2 : 1)
 topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
                   const int* __restrict__ row_len, int max_len, int k, int* __restrict__ idx,
                   long long ld_idx, const int* __restrict__ row_mask, int idx_offset,
@@ -375,32 +390,32 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
     }
     int* out = idx + (long long)r * ld_idx;
     if (n <= k) {  // every valid key is selected
-        for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i + idx_offset : -1;
+        for (int i = threadIdx.x; i < k; i += TopkCfg<T>::kThreads) out[i] = i < n ? i + idx_offset : -1;
         return;
     }
     const float* row = scores + (long long)r * ld;
     const int nwords = (n + 31) >> 5;
-    for (int i = threadIdx.x; i < nwords; i += kThreads) tie[i] = 0u;
+    for (int i = threadIdx.x; i < nwords; i += TopkCfg<T>::kThreads) tie[i] = 0u;
     __syncthreads();
 
     // ---- provisional threshold from a sample of the row ----
     uint32_t tau0 = 0u;
-    const uint32_t slice0 = (uint32_t)warp * kSlice;
-    if (n > kNoSampleMax) {
+    const uint32_t slice0 = (uint32_t)warp * TopkCfg<T>::kSlice;
+    if (n > TopkCfg<T>::kNoSampleMax) {
         const int nchunks = (n + 31) >> 5;
         const int stride = max(16, (nchunks + kSampleChunks - 1) / kSampleChunks);
         const int nsamp = (nchunks + stride - 1) / stride;  // sampled chunks, <= 256
-        float xs[kSampleChunksPerWarp];
+        float xs[TopkCfg<T>::kSampleChunksPerWarp];
 #pragma unroll
-        for (int i = 0; i < kSampleChunksPerWarp; ++i) {
-            const int j = warp + i * kWarps;
+        for (int i = 0; i < TopkCfg<T>::kSampleChunksPerWarp; ++i) {
+            const int j = warp + i * TopkCfg<T>::kWarps;
             const int sidx = j * stride * 32 + lane;
             xs[i] = (j < nsamp && sidx < n) ? __ldg(row + sidx) : 0.f;
         }
         uint32_t cnt = 0;
 #pragma unroll
-        for (int i = 0; i < kSampleChunksPerWarp; ++i) {
-            const int j = warp + i * kWarps;
+        for (int i = 0; i < TopkCfg<T>::kSampleChunksPerWarp; ++i) {
+            const int j = warp + i * TopkCfg<T>::kWarps;
             const int sidx = j * stride * 32 + lane;
             const bool in = j < nsamp && sidx < n;
             const unsigned m = __ballot_sync(0xffffffffu, in);
@@ -411,22 +426,22 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
         __syncthreads();
         uint32_t m = 0;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) m += sh.wcount[w];
+        for (int w = 0; w < TopkCfg<T>::kWarps; ++w) m += sh.wcount[w];
         // rank in the sample whose key should leave >= k keys of the row above it
         const float expect = (float)k * (float)m / (float)n;
         uint32_t rank = (uint32_t)ceilf(expect + 3.f * sqrtf(expect)) + 2u;
         if (rank > m) rank = m;
         uint32_t dummy;
-        tau0 = slice_radix_select(sh, rank, false, &dummy);
+        tau0 = slice_radix_select<T>(sh, rank, false, &dummy);
     }
 
     // ---- one pass: every key >= tau0 becomes a candidate in this warp's slice ----
     uint32_t cnt = 0;
-    for (int base = warp * 128; base < n; base += kWarps * 128 * kUnroll) {
+    for (int base = warp * 128; base < n; base += TopkCfg<T>::kWarps * 128 * kUnroll) {
         float4 v[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int s0 = base + u * kWarps * 128 + 4 * lane;
+            const int s0 = base + u * TopkCfg<T>::kWarps * 128 + 4 * lane;
             if (s0 + 3 < n) {
                 v[u] = __ldg(reinterpret_cast<const float4*>(row + s0));
             } else {
@@ -438,7 +453,7 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int s0 = base + u * kWarps * 128 + 4 * lane;
+            const int s0 = base + u * TopkCfg<T>::kWarps * 128 + 4 * lane;
             const float xv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -447,7 +462,7 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
                 const unsigned m = __ballot_sync(0xffffffffu, take);
                 if (take) {
                     const uint32_t p = cnt + __popc(m & lanemask_lt());
-                    if (p < (uint32_t)kSlice) {
+                    if (p < (uint32_t)TopkCfg<T>::kSlice) {
                         sh.cand_key[slice0 + p] = key;
                         sh.cand_idx[slice0 + p] = s0 + e;
                     }
@@ -456,20 +471,20 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
             }
         }
     }
-    for (int i = threadIdx.x; i < nwords; i += kThreads) sel[i] = 0u;
+    for (int i = threadIdx.x; i < nwords; i += TopkCfg<T>::kThreads) sel[i] = 0u;
     __syncthreads();  // everyone is past the sample select before wcount is rewritten
     if (lane == 0) sh.wcount[warp] = cnt;
     __syncthreads();
     uint32_t ncand = 0;
     bool overflow = false;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < TopkCfg<T>::kWarps; ++w) {
         ncand += sh.wcount[w];
-        overflow |= sh.wcount[w] > (uint32_t)kSlice;
+        overflow |= sh.wcount[w] > (uint32_t)TopkCfg<T>::kSlice;
     }
     uint32_t need;
     if (!overflow && ncand >= (uint32_t)k) {
-        const uint32_t tau = slice_radix_select(sh, (uint32_t)k, true, &need);
+        const uint32_t tau = slice_radix_select<T>(sh, (uint32_t)k, true, &need);
         for (int c = lane; c < (int)cnt; c += 32) {
             const uint32_t key = sh.cand_key[slice0 + c];
             const int sidx = sh.cand_idx[slice0 + c];
@@ -477,11 +492,11 @@ topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
             else if (key == tau) atomicOr(&tie[sidx >> 5], 1u << (sidx & 31));
         }
     } else {
-        need = exact_row_select(sh, row, n, k, sel, tie);
+        need = exact_row_select<T>(sh, row, n, k, sel, tie);
     }
     __syncthreads();
 
-    trim_ties_and_compact(sh, sel, tie, nwords, need, k, out, idx_offset);
+    trim_ties_and_compact<T>(sh, sel, tie, nwords, need, k, out, idx_offset);
 }
 
 
@@ -546,7 +561,8 @@ topk_threshold_kernel(const float* __restrict__ sample, long long ld_sample, int
 // k-th largest key and every key equal to it are among them.  Rows whose lists overflowed
 // or with fewer than k candidates are flagged for the dense fallback (fb_row[r] = 1,
 // *fb_any = 1) and left unwritten.
-__global__ void __launch_bounds__(kThreads, 2)
+template <int T>
+__global__ void __launch_bounds__(T, T <= 512 ? 2 : 1)
 topk_candidates_kernel(const uint2* __restrict__ cand, const uint32_t* __restrict__ ccount,
                        int cq, int nchunk_max, int q_begin, int max_len, int k,
                        int* __restrict__ idx, long long ld_idx, int* __restrict__ fb_row,
@@ -563,11 +579,11 @@ topk_candidates_kernel(const uint2* __restrict__ cand, const uint32_t* __restric
     int* out = idx + (long long)r * ld_idx;
     if (n <= k) {  // every valid key is selected
         if (threadIdx.x == 0) fb_row[r] = 0;
-        for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
+        for (int i = threadIdx.x; i < k; i += TopkCfg<T>::kThreads) out[i] = i < n ? i : -1;
         return;
     }
     const int nwords = (n + 31) >> 5;
-    for (int i = threadIdx.x; i < nwords; i += kThreads) sel[i] = 0u;
+    for (int i = threadIdx.x; i < nwords; i += TopkCfg<T>::kThreads) sel[i] = 0u;
     // the row's lists (chunk, quadrant) are dealt round-robin to the warps, each appending
     // into its slice of the candidate buffer
     const int nlists = ((n + 4095) >> 12) * 4;
@@ -575,14 +591,14 @@ topk_candidates_kernel(const uint2* __restrict__ cand, const uint32_t* __restric
     const uint2* lrow = cand + (long long)r * nchunk_max * 4 * cq;
     uint32_t filled = 0;
     bool over = false;
-    for (int l = warp; l < nlists; l += kWarps) {
+    for (int l = warp; l < nlists; l += TopkCfg<T>::kWarps) {
         const uint32_t len = __ldg(crow + l);
-        if (len > (uint32_t)cq || filled + len > (uint32_t)kSlice) { over = true; break; }
+        if (len > (uint32_t)cq || filled + len > (uint32_t)TopkCfg<T>::kSlice) { over = true; break; }
         const uint2* src = lrow + (long long)l * cq;
         for (uint32_t i = lane; i < len; i += 32) {
             const uint2 v = __ldg(src + i);
-            sh.cand_key[warp * kSlice + filled + i] = v.x;
-            sh.cand_idx[warp * kSlice + filled + i] = (int)v.y;
+            sh.cand_key[warp * TopkCfg<T>::kSlice + filled + i] = v.x;
+            sh.cand_idx[warp * TopkCfg<T>::kSlice + filled + i] = (int)v.y;
         }
         filled += len;
     }
@@ -591,7 +607,7 @@ topk_candidates_kernel(const uint2* __restrict__ cand, const uint32_t* __restric
     uint32_t c = 0;
     bool fail = false;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < TopkCfg<T>::kWarps; ++w) {
         const uint32_t v = sh.wcount[w];
         fail |= v == 0xFFFFFFFFu;
         c += v;
@@ -600,11 +616,11 @@ topk_candidates_kernel(const uint2* __restrict__ cand, const uint32_t* __restric
         if (threadIdx.x == 0) { fb_row[r] = 1; atomicExch(fb_any, 1); }
         return;
     }
-    for (int i = threadIdx.x; i < nwords; i += kThreads) tie[i] = 0u;
+    for (int i = threadIdx.x; i < nwords; i += TopkCfg<T>::kThreads) tie[i] = 0u;
     uint32_t need;
-    const uint32_t tau = slice_radix_select(sh, (uint32_t)k, true, &need);
+    const uint32_t tau = slice_radix_select<T>(sh, (uint32_t)k, true, &need);
     {
-        const int lo = warp * kSlice, cnt = (int)sh.wcount[warp];
+        const int lo = warp * TopkCfg<T>::kSlice, cnt = (int)sh.wcount[warp];
         for (int i = lane; i < cnt; i += 32) {
             const uint32_t key = sh.cand_key[lo + i];
             const int s = sh.cand_idx[lo + i];
@@ -614,7 +630,7 @@ topk_candidates_kernel(const uint2* __restrict__ cand, const uint32_t* __restric
     }
     __syncthreads();
     if (threadIdx.x == 0) fb_row[r] = 0;
-    trim_ties_and_compact(sh, sel, tie, nwords, need, k, out);
+    trim_ties_and_compact<T>(sh, sel, tie, nwords, need, k, out);
 }
 }  // namespace
 
@@ -628,12 +644,15 @@ cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin
                         cudaStream_t stream, const DevCtx& ctx, const int* row_mask,
                         int idx_offset) {
     const size_t smem = topk_smem_bytes(max_len);
-    cudaError_t e = cudaFuncSetAttribute(topk_radix_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // fewer rows than SMs (a decode batch): one 1024-thread CTA per row shortens each
+    // row's chain of block-wide phases; otherwise two 512-thread CTAs per SM
+    const bool wide = rows < ctx.num_sms;
+    auto kernel = wide ? topk_radix_kernel<1024> : topk_radix_kernel<512>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    topk_radix_kernel<<<rows, kThreads, smem, stream>>>(scores, ld, q_begin, row_len, max_len, k,
-                                                        idx, ld_idx, row_mask, idx_offset,
-                                                        ctx.err);
+    kernel<<<rows, wide ? 1024 : 512, smem, stream>>>(scores, ld, q_begin, row_len, max_len, k,
+                                                       idx, ld_idx, row_mask, idx_offset, ctx.err);
     count_launch(DSA_KERNEL_TOPK);
     return cudaGetLastError();
 }
@@ -655,10 +674,10 @@ cudaError_t launch_topk_candidates(const uint2* cand, const uint32_t* ccount, in
                                    int* idx, long long ld_idx, int* fb_row, int* fb_any,
                                    cudaStream_t stream) {
     const size_t smem = topk_smem_bytes(max_len);
-    cudaError_t e = cudaFuncSetAttribute(topk_candidates_kernel,
+    cudaError_t e = cudaFuncSetAttribute(topk_candidates_kernel<512>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    topk_candidates_kernel<<<rows, kThreads, smem, stream>>>(cand, ccount, cq, nchunk_max,
+    topk_candidates_kernel<512><<<rows, 512, smem, stream>>>(cand, ccount, cq, nchunk_max,
                                                              q_begin, max_len, k, idx, ld_idx,
                                                              fb_row, fb_any);
     count_launch(DSA_KERNEL_TOPK);
