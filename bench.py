@@ -44,6 +44,10 @@ def parse_args(argv=None):
                     help="prefill: the T=65536 headline; decode: 64 sequences x 32768 paged "
                          "tokens; stack: the 27-layer FSS x 9 IndexCache stack at T=16384; "
                          "varlen: 16 packed prompts of 512..8192 tokens in one batch")
+    ap.add_argument("--shard", choices=["sequences", "rows"], default="sequences",
+                    help="N>1: sequences = one sequence per rank (weak scaling); rows = the "
+                         "query rows of one T-token prefill split over the ranks (strong "
+                         "scaling, one all-gather of keys and latent rows per step)")
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
                     help="latent cache: bf16, or E4M3 codes times one fp32 scale")
     ap.add_argument("--window-rows", type=int, default=0,
@@ -510,6 +514,74 @@ def run_native(args, rank, world, local_rank):
     return result
 
 
+def run_rows(args, rank, world, local_rank):
+    """One T-token prefill with its query rows split over the ranks (zig-zag blocks):
+    each step all-gathers every rank's token shard of indexer keys and latent rows, then
+    runs indexer + top-k + sparse MLA for the rank's own query blocks."""
+    import torch
+    import sparse_attention_17_b200 as dsa
+    from sparse_attention_17_b200 import inputs as G
+    from sparse_attention_17_b200 import sharding as SH
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    T, k = args.T, args.topk
+    host = make_inputs(T, k, seed=0)  # one sequence: the same inputs on every rank
+    x = {n: host[n].to(dev) for n in ("q_idx", "w", "q")}
+    s0, ns = SH.token_shard(T, world, rank)
+    k_local = host["k_idx"][s0:s0 + ns].to(dev)
+    kv_local = host["kv"][s0:s0 + ns].to(dev)
+    k_full = torch.empty((T, 64), dtype=torch.bfloat16, device=dev)
+    kv_full = torch.empty((T, 576), dtype=torch.bfloat16, device=dev)
+    blocks = SH.zigzag_blocks(T, world, rank)
+    ld = (T + 3) // 4 * 4
+    rw = max(16, dsa.layer_stack_workspace_size(T, args.window_rows) // (4 * ld)) // 16 * 16
+    scores = torch.empty((rw, ld), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    out = torch.empty((T, 16, 512), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        SH.all_gather_rows(k_local, k_full)
+        SH.all_gather_rows(kv_local, kv_full)
+        for q0, rows in blocks:
+            for w0 in range(q0, q0 + rows, rw):
+                wr = min(rw, q0 + rows - w0)
+                dsa.indexer_scores(x["q_idx"], k_full, x["w"], scores, w0, wr)
+                dsa.topk_select(scores, k, idx[w0:w0 + wr], q_begin=w0, rows=wr)
+            dsa.sparse_mla_fwd(x["q"][q0:q0 + rows], kv_full, idx[q0:q0 + rows],
+                               out[q0:q0 + rows], G.SCALE_MLA)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
+    errs = dsa.check_device_errors()
+    if rank != 0:
+        return None
+    scored, attended = SH.pair_counts(blocks, k)
+    return {"metric": METRIC, "value": round(T / (ms / 1e3), 1), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"dsa_prefill_T{T}_top{k}", "T": T, "topk": k,
+                       "parallelism": f"query rows x{world} (zig-zag blocks, all-gather of "
+                                      "k_idx and latent rows per step)",
+                       "rank0_blocks": blocks, "rank0_scored_pairs": scored,
+                       "rank0_attended_keys": attended},
+            "clocks": clk.summary(), "device_error_bits": errs}
+
+
 def _timed(step, steps, warmup, stream):
     """Device time of `steps` calls of step() after `warmup` calls (CUDA events)."""
     import torch
@@ -731,6 +803,8 @@ def main(argv=None):
             res = run_stack(args, local_rank) if rank == 0 else None
         elif args.workload == "varlen":
             res = run_varlen(args, local_rank) if rank == 0 else None
+        elif args.shard == "rows":
+            res = run_rows(args, rank, world, local_rank)
         else:
             res = run_native(args, rank, world, local_rank)
     finally:
