@@ -87,7 +87,9 @@ const char* dsa_status_string(int status);
 /* Detail of the last error returned on the calling host thread ("" if none). */
 const char* dsa_last_error(void);
 
-/* ABI version of this header: (major << 16) | minor. */
+/* ABI version of this header: (major << 16) | minor.  1.1 added dsa_index_select,
+ * dsa_index_varlen, the fp8 cache calls, dsa_selftest_wait_timeout and
+ * DSA_KERNEL_QUANTIZE. */
 int dsa_version(void);
 
 /*

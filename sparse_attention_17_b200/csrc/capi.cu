@@ -140,7 +140,7 @@ const char* dsa_status_string(int status) {
 
 const char* dsa_last_error(void) { return g_last_error; }
 
-int dsa_version(void) { return (1 << 16) | 0; }
+int dsa_version(void) { return (1 << 16) | 1; }
 
 dsa_status dsa_indexer_scores(int dtype, int mode, const void* q_idx, const void* k_idx,
                               const float* w, int H_I, int D_I, int q_begin, int rows, int S,
