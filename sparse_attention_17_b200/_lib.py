@@ -111,6 +111,16 @@ def _need(t, dtype, ndim, name):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _scratch(workspace) -> tuple[int | None, int]:
+    """(pointer, bytes) of an optional workspace: a contiguous CUDA tensor of any dtype."""
+    if workspace is None:
+        return None, 0
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda \
+            or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
 def _dt(t) -> int:
     if t.dtype == torch.bfloat16:
         return DSA_BF16
@@ -190,8 +200,7 @@ def index_select(q_idx, k_idx, w, idx, k: int, workspace, q_begin: int = 0,
         rows = q_idx.shape[0] - q_begin
     _check(lib.dsa_index_select(q_idx.data_ptr(), k_idx.data_ptr(), w.data_ptr(), q_idx.shape[1],
                                 q_idx.shape[2], q_begin, rows, k_idx.shape[0], k, idx.data_ptr(),
-                                idx.stride(0), workspace.data_ptr(),
-                                workspace.numel() * workspace.element_size(), _stream()))
+                                idx.stride(0), *_scratch(workspace), _stream()))
 
 
 def sparse_mla_workspace_size(num_q: int, k_sel: int, decode: bool, H: int = 16,
@@ -214,9 +223,7 @@ def sparse_mla_fwd(q, kv, idx, out, scale: float, lse=None, v=None, page_table=N
         _need(lse, torch.float32, 2, "lse")
     num_q, H, D_qk = q.shape
     k_sel = idx.shape[1]
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    ws_ptr, ws_bytes = _scratch(workspace)
     if v is not None:  # MHA
         _need(kv, q.dtype, 3, "k")
         _need(v, q.dtype, 3, "v")
@@ -259,9 +266,7 @@ def sparse_mla_fp8_fwd(q, kv, kv_scale: float, idx, out, scale: float, lse=None,
     num_q, H, D_qk = q.shape
     D_v = out.shape[2]
     k_sel = idx.shape[1]
-    ws_ptr, ws_bytes = None, 0
-    if workspace is not None:
-        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    ws_ptr, ws_bytes = _scratch(workspace)
     if page_table is None:
         _need(kv, torch.uint8, 2, "kv")
         _check(lib.dsa_sparse_mla_fp8_fwd(DSA_PREFILL, num_q, H, D_qk, D_v, scale, kv_scale,
@@ -302,8 +307,7 @@ def index_varlen(q_idx, k_idx, w, seq_start, seq_len, k: int, idx, workspace) ->
                                 q_idx.shape[2], q_idx.shape[0], n,
                                 ctypes.cast(starts, ctypes.c_void_p),
                                 ctypes.cast(lens, ctypes.c_void_p), k, idx.data_ptr(),
-                                idx.stride(0), workspace.data_ptr(),
-                                workspace.numel() * workspace.element_size(), _stream()))
+                                idx.stride(0), *_scratch(workspace), _stream()))
 
 
 def selftest_wait_timeout(gave_up) -> None:
@@ -315,10 +319,10 @@ def selftest_wait_timeout(gave_up) -> None:
 def latent_quantize_fp8(src, kv_scale: float, dst) -> None:
     """dsa_latent_quantize_fp8: dst (uint8, same shape) = E4M3(src (bf16) / kv_scale)."""
     lib = load()
-    if src.dtype != torch.bfloat16 or dst.dtype != torch.uint8:
-        raise TypeError("src must be bfloat16 and dst uint8")
-    if not (src.is_contiguous() and dst.is_contiguous()) or src.numel() != dst.numel():
-        raise ValueError("src and dst must be contiguous with the same number of elements")
+    _need(src, torch.bfloat16, None, "src")
+    _need(dst, torch.uint8, None, "dst")
+    if src.numel() != dst.numel():
+        raise ValueError("src and dst must have the same number of elements")
     _check(lib.dsa_latent_quantize_fp8(src.data_ptr(), src.numel(), kv_scale, dst.data_ptr(),
                                        _stream()))
 
@@ -356,12 +360,14 @@ def layer_stack(pattern: str, layers: list[dict], idx_buf, workspace, topk: int,
     w = ptrs("w", layers)
     q = ptrs("q", layers)
     kv = ptrs("kv", layers)
+    for l, x in enumerate(lses or []):
+        if x is not None:
+            _need(x, torch.float32, 2, f"lses[{l}]")
     out = arr(*[o.data_ptr() for o in outs])
     lse = arr(*[(x.data_ptr() if x is not None else None) for x in lses]) if lses else None
-    ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib.dsa_layer_stack(pattern.encode(), n, T, topk, 16, 64, 16, 576, 512, scale,
                                q_idx, k_idx, w, q, kv, out, lse, idx_buf.data_ptr(),
-                               workspace.data_ptr(), ws_bytes, _stream()))
+                               *_scratch(workspace), _stream()))
 
 
 def pattern_from_freq(freq: int, num_layers: int) -> str:

@@ -218,3 +218,14 @@ def test_index_select_rejects_and_sizes(lib):
     a = lib.dsa_index_select_workspace_size(16, 8192)
     assert 0 < a < lib.dsa_index_select_workspace_size(32, 8192) < lib.dsa_index_select_workspace_size(32, 65536)
     assert lib.dsa_index_select_workspace_size(0, 8192) == 0
+
+
+def test_binding_refuses_host_tensors_before_the_library():
+    """Host (CPU) tensors never reach a kernel: the binding raises first."""
+    import torch
+    with pytest.raises(ValueError):
+        dsa.latent_quantize_fp8(torch.zeros(8, dtype=torch.bfloat16), 0.01,
+                                torch.zeros(8, dtype=torch.uint8))
+    with pytest.raises(ValueError):
+        _lib._scratch(torch.zeros(16))
+    assert _lib._scratch(None) == (None, 0)
