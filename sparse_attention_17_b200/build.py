@@ -2,6 +2,7 @@
 
     python -m sparse_attention_17_b200.build          # incremental
     python -m sparse_attention_17_b200.build --force  # rebuild
+    python -m sparse_attention_17_b200.build --force --nvtx  # with NVTX ranges (tracing)
 """
 from __future__ import annotations
 
@@ -38,8 +39,9 @@ def _stale() -> bool:
     return any(p.stat().st_mtime > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> Path:
-    """Compiles every kernel file into libdsa.so next to this module (sm_100a only)."""
+def build(force: bool = False, verbose: bool = False, nvtx: bool = False) -> Path:
+    """Compiles every kernel file into libdsa.so next to this module (sm_100a only).  With
+    nvtx, the host side marks layers and index windows as NVTX ranges for timelines."""
     if not force and not _stale():
         return LIB
     build_dir = PKG / "_build"
@@ -48,7 +50,8 @@ def build(force: bool = False, verbose: bool = False) -> Path:
     for src in sources():
         obj = build_dir / (src.stem + ".o")
         cmd = [nvcc(), *ARCH, "-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC",
-               "-Xptxas", "-v" if verbose else "-O3", f"-I{INCLUDE}", "-c", str(src), "-o", str(obj)]
+               "-Xptxas", "-v" if verbose else "-O3", f"-I{INCLUDE}",
+               *(["-DDSA_NVTX=1"] if nvtx else []), "-c", str(src), "-o", str(obj)]
         subprocess.run(cmd, check=True)
         objs.append(str(obj))
     tmp = LIB.with_suffix(f".so.{os.getpid()}.tmp")
@@ -61,8 +64,9 @@ def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true", help="print ptxas register/smem usage")
+    ap.add_argument("--nvtx", action="store_true", help="NVTX ranges per layer and window")
     a = ap.parse_args(argv)
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, nvtx=a.nvtx))
     return 0
 
 

@@ -13,6 +13,10 @@
 #include "dsa_common.cuh"
 #include "launch.h"
 
+#if defined(DSA_NVTX) && DSA_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
+
 namespace dsa {
 
 // Per-device error word: kernels OR DSA_DEVERR_* bits into it; dsa_check_device_errors
@@ -112,6 +116,25 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
 size_t topk_smem_bytes(int max_len);
 
 // Validation shared by the calls.
+// Tracing: an NVTX range for the lifetime of the object when the library is built with
+// -DDSA_NVTX=1 (build.py --nvtx), so that timelines show each layer and index window; an
+// empty object otherwise.
+struct TraceRange {
+#if defined(DSA_NVTX) && DSA_NVTX
+    explicit TraceRange(const char* fmt, ...) {
+        char name[96];
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(name, sizeof name, fmt, ap);
+        va_end(ap);
+        nvtxRangePushA(name);
+    }
+    ~TraceRange() { nvtxRangePop(); }
+#else
+    explicit TraceRange(const char*, ...) {}
+#endif
+};
+
 dsa_status check_stream_device(DevCtx* ctx) {
     cudaError_t e = get_dev_ctx(ctx);
     if (e == cudaErrorNoKernelImageForDevice)
@@ -640,9 +663,11 @@ dsa_status dsa_layer_stack(const char* pattern, int num_layers, int T, int topk,
     if (rw > 16) rw = rw / 16 * 16;  // whole 16-query blocks per window
     float* scores = static_cast<float*>(workspace);
     for (int l = 0; l < num_layers; ++l) {
+        TraceRange layer_range("dsa layer %d (%c)", l, pattern[l]);
         if (pattern[l] == 'F') {
             for (long long q0 = 0; q0 < T; q0 += rw) {
                 const int rows = (int)((T - q0) < rw ? (T - q0) : rw);
+                TraceRange window_range("dsa index window %lld+%d", q0, rows);
                 dsa_status st = dsa_indexer_scores(DSA_BF16, DSA_PREFILL, q_idx[l], k_idx[l], w[l],
                                                    H_I, D_I, (int)q0, rows, T, nullptr, 0, 0,
                                                    nullptr, scores, ld, stream);
