@@ -224,7 +224,7 @@ size_t dsa_sparse_mla_workspace_size(int mode, int num_q, int H, int D_v, int k_
  * All calls share the one array: calls that overlap on the GPU (other streams, other host
  * threads) race and must be serialised by the caller.  Each call overwrites the parts of
  * the array it uses, so nothing has to be cleared between calls.  Errors: as for
- * dsa_sparse_mla_fwd (dsa_last_error() is not set by this call).
+ * dsa_sparse_mla_fwd; dsa_last_error() describes the failure.
  */
 dsa_status dsa_sparse_mla_decode_noalloc(int num_q, int H, int D_qk, int D_v, float scale,
                                          const void* q, const void* kv, long long kv_rows,

@@ -11,6 +11,7 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 from pathlib import Path
 
 PKG = Path(__file__).resolve().parent
@@ -46,14 +47,17 @@ def build(force: bool = False, verbose: bool = False, nvtx: bool = False) -> Pat
         return LIB
     build_dir = PKG / "_build"
     build_dir.mkdir(exist_ok=True)
-    objs = []
+    objs, cmds = [], []
     for src in sources():
         obj = build_dir / (src.stem + ".o")
-        cmd = [nvcc(), *ARCH, "-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC",
-               "-Xptxas", "-v" if verbose else "-O3", f"-I{INCLUDE}",
-               *(["-DDSA_NVTX=1"] if nvtx else []), "-c", str(src), "-o", str(obj)]
-        subprocess.run(cmd, check=True)
+        cmds.append([nvcc(), *ARCH, "-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC",
+                     "-Xptxas", "-v" if verbose else "-O3", f"-I{INCLUDE}",
+                     *(["-DDSA_NVTX=1"] if nvtx else []), "-c", str(src), "-o", str(obj)])
         objs.append(str(obj))
+    # the kernel files compile independently: one nvcc per file, in parallel
+    with ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 1)) as pool:
+        for fut in [pool.submit(subprocess.run, c, check=True) for c in cmds]:
+            fut.result()
     tmp = LIB.with_suffix(f".so.{os.getpid()}.tmp")
     subprocess.run([nvcc(), *ARCH, "-shared", "-o", str(tmp), *objs], check=True)
     os.replace(tmp, LIB)

@@ -98,6 +98,16 @@ void count_launch(int kind) {
     if (kind >= 0 && kind < DSA_KERNEL_KINDS) g_launches[kind].fetch_add(1);
 }
 
+void clear_last_error() { g_last_error[0] = 0; }
+
+dsa_status fail_with(dsa_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                        uint64_t row_pitch_bytes, uint32_t box_rows, uint32_t box_cols) {
     EncodeTiledFn fn = encode_fn();
@@ -112,8 +122,6 @@ bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
-
-size_t topk_smem_bytes(int max_len);
 
 // Validation shared by the calls.
 // Tracing: an NVTX range for the lifetime of the object when the library is built with

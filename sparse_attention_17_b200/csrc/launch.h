@@ -24,6 +24,11 @@ cudaError_t get_dev_ctx(DevCtx* ctx);
 // Counts one launch of a kernel family (dsa_launch_count).
 void count_launch(int kind);
 
+// The calling thread's message for dsa_last_error: cleared on entry to every call, set
+// (printf-style) with the status a call returns on failure.
+void clear_last_error();
+dsa_status fail_with(dsa_status st, const char* fmt, ...);
+
 // Builds a 2-D bf16 tensor map (rows x cols, row pitch in bytes) with a box of
 // box_rows x box_cols and 128-byte swizzle.  Returns false if the driver rejects it.
 bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,

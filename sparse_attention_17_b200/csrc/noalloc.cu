@@ -59,24 +59,31 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(
     long long kv_rows, const int* page_table, int max_pages, int page_size,
     const int* seq_lens, const int* idx, int k_sel, long long ld_idx, void* out, float* lse,
     dsa_stream_t stream) {
+    clear_last_error();
     auto aligned = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
     if (!q || !kv || !idx || !out || !page_table || !seq_lens)
-        return DSA_ERR_INVALID_ARG;
+        return fail_with(DSA_ERR_INVALID_ARG, "null tensor pointer");
     if (!aligned(q) || !aligned(kv) || !aligned(idx) || !aligned(out) || (lse && !aligned(lse)))
-        return DSA_ERR_INVALID_ARG;
+        return fail_with(DSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
     if (num_q < 0 || kv_rows <= 0 || k_sel <= 0 || ld_idx < k_sel || page_size <= 0 ||
         max_pages <= 0 || kv_rows % page_size || !(scale > 0.f))
-        return DSA_ERR_INVALID_ARG;
+        return fail_with(DSA_ERR_INVALID_ARG, "bad sizes or scale");
     if (H != 16 || D_qk != 576 || D_v != 512 || k_sel > 2048 || (k_sel & 3) || (ld_idx & 3))
-        return DSA_ERR_UNSUPPORTED;
+        return fail_with(DSA_ERR_UNSUPPORTED,
+                         "absorbed MLA only: H=16, 576/512, k_sel <= 2048, multiples of 4");
     if (num_q == 0) return DSA_OK;
-    if (num_q > kMaxUnits) return DSA_ERR_UNSUPPORTED;  // even one split per sequence won't fit
+    if (num_q > kMaxUnits)  // even one split per sequence would not fit the array
+        return fail_with(DSA_ERR_UNSUPPORTED, "at most %d sequences per call, got %d", kMaxUnits,
+                         num_q);
     DevCtx ctx;
     cudaError_t e = get_dev_ctx(&ctx);
-    if (e == cudaErrorNoKernelImageForDevice) return DSA_ERR_UNSUPPORTED;
-    if (e != cudaSuccess) return DSA_ERR_CUDA;
+    if (e == cudaErrorNoKernelImageForDevice)
+        return fail_with(DSA_ERR_UNSUPPORTED, "this library is built for sm_100a (B200) only");
+    if (e != cudaSuccess) return fail_with(DSA_ERR_CUDA, "device query: %s", cudaGetErrorString(e));
     void* scratch = nullptr;
-    if (scratch_address(&scratch) != cudaSuccess) return DSA_ERR_CUDA;
+    e = scratch_address(&scratch);
+    if (e != cudaSuccess)
+        return fail_with(DSA_ERR_CUDA, "scratch array address: %s", cudaGetErrorString(e));
     // as many splits as the usual path would take, capped by what the array holds (a
     // trailing split left without keys writes a zero partial with log-sum-exp -inf, which
     // the merge ignores)
@@ -90,8 +97,9 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(
     e = launch_sparse_mla_mma(static_cast<const __nv_bfloat16*>(q), kv, false, 1.f, kv_rows, page_table,
                                max_pages, page_size, seq_lens, idx, k_sel, ld_idx, num_q, scale,
                                splits, nullptr, nullptr, o_part, lse_part, cs, ctx);
-    if (e != cudaSuccess) return DSA_ERR_CUDA;
+    if (e != cudaSuccess) return fail_with(DSA_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
     e = launch_mla_combine(o_part, lse_part, num_q, splits, static_cast<__nv_bfloat16*>(out), lse,
                            cs);
-    return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+    if (e != cudaSuccess) return fail_with(DSA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+    return DSA_OK;
 }

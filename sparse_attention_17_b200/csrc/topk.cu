@@ -1,28 +1,15 @@
-// topk.cu -- per-row top-k of fp32 indexer scores by radix selection (no sort).
+// topk.cu -- exact top-k among the candidate lists of the filtered index selection
+// (dsa_index_select): per-row thresholds from sampled scores, then the exact top-k among
+// the keys the filtered indexer kept.  The dense per-row top-k is in topk_stream.cu.
 //
 // Selection rule (DSA ablation card, "Attention" bullet and closing note): the k largest
 // of the row's n valid scores, equal scores resolved towards the lower key index; if
 // n <= k every key is selected.  Output: the selected key positions in ascending order,
 // then -1 padding.
 //
-// One CTA per row: 512 threads, or 1024 when the launch has fewer rows than the GPU has
-// SMs (a decode batch).  Scores map to order-preserving uint32 keys.  Each warp owns a
-// slice of the shared candidate buffer (512 entries, or 256 with 1024 threads), so
-// candidates are appended with a ballot and a popcount and no shared atomics.
-// Fast path (one read of the row):
-//   sample  every 16th 32-key chunk of the row (at most 256 chunks, all loads in flight
-//           at once) goes to the slices; a two-round (12 + 12 bit) radix select there
-//           gives a provisional threshold tau0 below the sample rank that corresponds to
-//           k plus a few standard deviations (rows of at most 8192 keys skip this:
-//           tau0 = the smallest key);
-//   gather  one pass with four 16-byte loads per thread in flight appends every key
-//           >= tau0 to the warp's slice (128-key chunks dealt round-robin to the warps);
-//   select  radix select (12 + 12 + 8 bits) among the candidates gives the k-th largest
-//           key tau; candidates above tau are selected, those equal to tau are ties.
-// If the candidates number fewer than k or more than a slice holds, the row is redone
-// exactly from global memory (histogram passes over the whole row).  Finally the first
-// `need` ties in index order are kept and a bitmap of the selection is compacted in index
-// order, which yields ascending indices without sorting.
+// Scores map to order-preserving uint32 keys.  Each warp owns a slice of the shared
+// candidate buffer, radix selection (12 + 12 + 8 bits) among the candidates gives the
+// k-th largest key, and a bitmap of the selection is compacted in index order.
 #include "dsa_common.cuh"
 #include "launch.h"
 
@@ -32,22 +19,15 @@ namespace {
 
 constexpr int kBins = 4096;
 constexpr int kCandCap = 8192;
-constexpr int kUnroll = 4;                 // 16-byte loads in flight per thread
 constexpr int kBM_SAMPLE = 128;            // keys per sampled tile (the indexer's tile)
 constexpr int kMaxWarps = 32;
-constexpr int kSampleChunks = kCandCap / 32;  // at most 256 sampled 32-key chunks
 
-// The block size: 512 threads (two CTAs per SM) when rows are plentiful, 1024 (one CTA
-// per SM) for launches with fewer rows than SMs, such as a decode batch.
+// The block size of the candidate selection (512 threads, two CTAs per SM).
 template <int T>
 struct TopkCfg {
     static constexpr int kThreads = T;
     static constexpr int kWarps = T / 32;
-    static constexpr int kStride = kWarps * 32;          // elements covered per iteration
     static constexpr int kSlice = kCandCap / kWarps;     // candidate entries of one warp
-    static constexpr int kSampleChunksPerWarp = kSampleChunks / kWarps;  // one slice
-    // rows this short make every key a candidate: each warp's 128-key chunks fit its slice
-    static constexpr int kNoSampleMax = (kSlice / 128) * 128 * kWarps;
     static_assert(kWarps <= kMaxWarps && kSlice % 128 == 0, "block size");
 };
 
@@ -61,12 +41,6 @@ struct TopkScratch {
     uint32_t found_bin;
     uint32_t found_above;
 };
-
-__device__ __forceinline__ uint32_t lanemask_lt() {
-    uint32_t m;
-    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-    return m;
-}
 
 // Adds 1 to hist[bin] for every lane with pred, one shared atomic per distinct bin.
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool pred) {
@@ -189,135 +163,6 @@ __device__ uint32_t slice_radix_select(TopkScratch& sh, uint32_t need, bool exac
     return tau;
 }
 
-// Exact selection from global memory (fallback): histogram passes over the whole row.
-// Fills sel (keys above the k-th largest) and tie (keys equal to it); returns how many
-// of the ties belong to the top k.  sel must be zero, tie zero on entry.
-template <int T>
-__device__ uint32_t exact_row_select(TopkScratch& sh, const float* __restrict__ row, int n,
-                                     int k, uint32_t* sel, uint32_t* tie) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // ---- pass 1: histogram of the top 12 key bits over the whole row ----
-    zero_hist<T>(sh, kBins);
-    if (threadIdx.x == 0) sh.cand_count = 0u;
-    __syncthreads();
-    for (int base = warp * 32; base < n; base += 4 * TopkCfg<T>::kStride) {
-        float x[4];
-        bool in[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int s = base + u * TopkCfg<T>::kStride + lane;
-            in[u] = s < n;
-            x[u] = in[u] ? __ldg(row + s) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) hist_add(sh.hist, float_order_key(x[u]) >> 20, in[u]);
-    }
-    __syncthreads();
-    find_bin<T>(sh, kBins, (uint32_t)k);
-    const uint32_t b1 = sh.found_bin;
-    uint32_t need = (uint32_t)k - sh.found_above;
-    const uint32_t cnt1 = sh.hist[b1];
-    __syncthreads();
-
-    uint32_t tau;
-    if (cnt1 <= (uint32_t)kCandCap) {
-        // ---- pass 2: definite selections to the bitmap, the b1 bucket to shared memory ----
-        for (int base = warp * 32; base < n; base += TopkCfg<T>::kStride) {
-            const int s = base + lane;
-            const bool in = s < n;
-            const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
-            const uint32_t hi = key >> 20;
-            const unsigned gt = __ballot_sync(0xffffffffu, in && hi > b1);
-            const bool eq = in && hi == b1;
-            const unsigned meq = __ballot_sync(0xffffffffu, eq);
-            if (lane == 0) sel[base >> 5] = gt;
-            if (meq) {
-                uint32_t pos0 = 0;
-                if (lane == 0) pos0 = atomicAdd(&sh.cand_count, (uint32_t)__popc(meq));
-                pos0 = __shfl_sync(0xffffffffu, pos0, 0);
-                if (eq) {
-                    const uint32_t p = pos0 + __popc(meq & lanemask_lt());
-                    sh.cand_key[p] = key;
-                    sh.cand_idx[p] = s;
-                }
-            }
-        }
-        zero_hist<T>(sh, kBins);
-        __syncthreads();
-        const int cnt = (int)sh.cand_count;
-        // ---- refine: bits 19..8 ----
-        for (int c0 = warp * 32; c0 < cnt; c0 += TopkCfg<T>::kStride) {
-            const int c = c0 + lane;
-            const bool in = c < cnt;
-            hist_add(sh.hist, in ? (sh.cand_key[c] >> 8) & 0xFFFu : 0u, in);
-        }
-        __syncthreads();
-        find_bin<T>(sh, kBins, need);
-        const uint32_t b2 = sh.found_bin;
-        need -= sh.found_above;
-        zero_hist<T>(sh, 256);
-        __syncthreads();
-        // ---- refine: bits 7..0 ----
-        const uint32_t pre = (b1 << 12) | b2;
-        for (int c0 = warp * 32; c0 < cnt; c0 += TopkCfg<T>::kStride) {
-            const int c = c0 + lane;
-            const uint32_t key = c < cnt ? sh.cand_key[c] : 0u;
-            const bool in = c < cnt && (key >> 8) == pre;
-            hist_add(sh.hist, key & 0xFFu, in);
-        }
-        __syncthreads();
-        find_bin<T>(sh, 256, need);
-        need -= sh.found_above;
-        tau = (pre << 8) | sh.found_bin;
-        for (int c = threadIdx.x; c < cnt; c += TopkCfg<T>::kThreads) {
-            const uint32_t key = sh.cand_key[c];
-            const int s = sh.cand_idx[c];
-            if (key > tau) atomicOr(&sel[s >> 5], 1u << (s & 31));
-            else if (key == tau) atomicOr(&tie[s >> 5], 1u << (s & 31));
-        }
-    } else {
-        // ---- the b1 bucket does not fit: refine from global memory ----
-        zero_hist<T>(sh, kBins);
-        __syncthreads();
-        for (int base = warp * 32; base < n; base += TopkCfg<T>::kStride) {
-            const int s = base + lane;
-            const bool in = s < n;
-            const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
-            hist_add(sh.hist, (key >> 8) & 0xFFFu, in && (key >> 20) == b1);
-        }
-        __syncthreads();
-        find_bin<T>(sh, kBins, need);
-        const uint32_t b2 = sh.found_bin;
-        need -= sh.found_above;
-        zero_hist<T>(sh, 256);
-        __syncthreads();
-        const uint32_t pre = (b1 << 12) | b2;
-        for (int base = warp * 32; base < n; base += TopkCfg<T>::kStride) {
-            const int s = base + lane;
-            const bool in = s < n;
-            const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
-            hist_add(sh.hist, key & 0xFFu, in && (key >> 8) == pre);
-        }
-        __syncthreads();
-        find_bin<T>(sh, 256, need);
-        need -= sh.found_above;
-        tau = (pre << 8) | sh.found_bin;
-        for (int base = warp * 32; base < n; base += TopkCfg<T>::kStride) {
-            const int s = base + lane;
-            const bool in = s < n;
-            const uint32_t key = float_order_key(in ? __ldg(row + s) : 0.f);
-            const unsigned gt = __ballot_sync(0xffffffffu, in && key > tau);
-            const unsigned eq = __ballot_sync(0xffffffffu, in && key == tau);
-            if (lane == 0) {
-                sel[base >> 5] = gt;
-                tie[base >> 5] = eq;
-            }
-        }
-    }
-    __syncthreads();
-    return need;
-}
-
 // Keeps the first `need` ties (tie bitmap) in index order, merges them into the selection
 // bitmap and writes the selected key positions in ascending order, then -1 up to k.
 template <int T>
@@ -362,143 +207,6 @@ __device__ void trim_ties_and_compact(TopkScratch& sh, uint32_t* sel, const uint
     }
     for (int i = (int)total + threadIdx.x; i < k; i += TopkCfg<T>::kThreads) out[i] = -1;
 }
-
-template <int T>
-__global__ void __launch_bounds__(T, T <= 512 ? 2 : 1)
-topk_radix_kernel(const float* __restrict__ scores, long long ld, int q_begin,
-                  const int* __restrict__ row_len, int max_len, int k, int* __restrict__ idx,
-                  long long ld_idx, const int* __restrict__ row_mask, int idx_offset,
-                  unsigned* __restrict__ err) {
-    if (row_mask != nullptr && row_mask[blockIdx.x] == 0) return;  // row not asked for
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    TopkScratch& sh = *reinterpret_cast<TopkScratch*>(smem_raw);
-    uint32_t* sel = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkScratch));
-    const int max_words = (max_len + 31) >> 5;
-    uint32_t* tie = sel + max_words;
-
-    const int r = blockIdx.x;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int n;
-    if (row_len != nullptr) {
-        n = row_len[r];
-        if (n < 0 || n > max_len) {
-            if (threadIdx.x == 0) atomicOr(err, DSA_DEVERR_INDEX_RANGE);
-            n = n < 0 ? 0 : max_len;
-        }
-    } else {
-        n = q_begin + r + 1;
-    }
-    int* out = idx + (long long)r * ld_idx;
-    if (n <= k) {  // every valid key is selected
-        for (int i = threadIdx.x; i < k; i += TopkCfg<T>::kThreads) out[i] = i < n ? i + idx_offset : -1;
-        return;
-    }
-    const float* row = scores + (long long)r * ld;
-    const int nwords = (n + 31) >> 5;
-    for (int i = threadIdx.x; i < nwords; i += TopkCfg<T>::kThreads) tie[i] = 0u;
-    __syncthreads();
-
-    // ---- provisional threshold from a sample of the row ----
-    uint32_t tau0 = 0u;
-    const uint32_t slice0 = (uint32_t)warp * TopkCfg<T>::kSlice;
-    if (n > TopkCfg<T>::kNoSampleMax) {
-        const int nchunks = (n + 31) >> 5;
-        const int stride = max(16, (nchunks + kSampleChunks - 1) / kSampleChunks);
-        const int nsamp = (nchunks + stride - 1) / stride;  // sampled chunks, <= 256
-        float xs[TopkCfg<T>::kSampleChunksPerWarp];
-#pragma unroll
-        for (int i = 0; i < TopkCfg<T>::kSampleChunksPerWarp; ++i) {
-            const int j = warp + i * TopkCfg<T>::kWarps;
-            const int sidx = j * stride * 32 + lane;
-            xs[i] = (j < nsamp && sidx < n) ? __ldg(row + sidx) : 0.f;
-        }
-        uint32_t cnt = 0;
-#pragma unroll
-        for (int i = 0; i < TopkCfg<T>::kSampleChunksPerWarp; ++i) {
-            const int j = warp + i * TopkCfg<T>::kWarps;
-            const int sidx = j * stride * 32 + lane;
-            const bool in = j < nsamp && sidx < n;
-            const unsigned m = __ballot_sync(0xffffffffu, in);
-            if (in) sh.cand_key[slice0 + cnt + __popc(m & lanemask_lt())] = float_order_key(xs[i]);
-            cnt += __popc(m);
-        }
-        if (lane == 0) sh.wcount[warp] = cnt;
-        __syncthreads();
-        uint32_t m = 0;
-#pragma unroll
-        for (int w = 0; w < TopkCfg<T>::kWarps; ++w) m += sh.wcount[w];
-        // rank in the sample whose key should leave >= k keys of the row above it
-        const float expect = (float)k * (float)m / (float)n;
-        uint32_t rank = (uint32_t)ceilf(expect + 3.f * sqrtf(expect)) + 2u;
-        if (rank > m) rank = m;
-        uint32_t dummy;
-        tau0 = slice_radix_select<T>(sh, rank, false, &dummy);
-    }
-
-    // ---- one pass: every key >= tau0 becomes a candidate in this warp's slice ----
-    uint32_t cnt = 0;
-    for (int base = warp * 128; base < n; base += TopkCfg<T>::kWarps * 128 * kUnroll) {
-        float4 v[kUnroll];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int s0 = base + u * TopkCfg<T>::kWarps * 128 + 4 * lane;
-            if (s0 + 3 < n) {
-                v[u] = __ldg(reinterpret_cast<const float4*>(row + s0));
-            } else {
-                v[u].x = s0 < n ? __ldg(row + s0) : 0.f;
-                v[u].y = s0 + 1 < n ? __ldg(row + s0 + 1) : 0.f;
-                v[u].z = s0 + 2 < n ? __ldg(row + s0 + 2) : 0.f;
-                v[u].w = 0.f;
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int s0 = base + u * TopkCfg<T>::kWarps * 128 + 4 * lane;
-            const float xv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const uint32_t key = float_order_key(xv[e]);
-                const bool take = s0 + e < n && key >= tau0;
-                const unsigned m = __ballot_sync(0xffffffffu, take);
-                if (take) {
-                    const uint32_t p = cnt + __popc(m & lanemask_lt());
-                    if (p < (uint32_t)TopkCfg<T>::kSlice) {
-                        sh.cand_key[slice0 + p] = key;
-                        sh.cand_idx[slice0 + p] = s0 + e;
-                    }
-                }
-                cnt += __popc(m);
-            }
-        }
-    }
-    for (int i = threadIdx.x; i < nwords; i += TopkCfg<T>::kThreads) sel[i] = 0u;
-    __syncthreads();  // everyone is past the sample select before wcount is rewritten
-    if (lane == 0) sh.wcount[warp] = cnt;
-    __syncthreads();
-    uint32_t ncand = 0;
-    bool overflow = false;
-#pragma unroll
-    for (int w = 0; w < TopkCfg<T>::kWarps; ++w) {
-        ncand += sh.wcount[w];
-        overflow |= sh.wcount[w] > (uint32_t)TopkCfg<T>::kSlice;
-    }
-    uint32_t need;
-    if (!overflow && ncand >= (uint32_t)k) {
-        const uint32_t tau = slice_radix_select<T>(sh, (uint32_t)k, true, &need);
-        for (int c = lane; c < (int)cnt; c += 32) {
-            const uint32_t key = sh.cand_key[slice0 + c];
-            const int sidx = sh.cand_idx[slice0 + c];
-            if (key > tau) atomicOr(&sel[sidx >> 5], 1u << (sidx & 31));
-            else if (key == tau) atomicOr(&tie[sidx >> 5], 1u << (sidx & 31));
-        }
-    } else {
-        need = exact_row_select<T>(sh, row, n, k, sel, tie);
-    }
-    __syncthreads();
-
-    trim_ties_and_compact<T>(sh, sel, tie, nwords, need, k, out, idx_offset);
-}
-
 
 // ---------------------------------------------------------------------------------------
 // Filtered selection (no dense score rows): thresholds from sampled scores, then the exact
@@ -637,24 +345,6 @@ topk_candidates_kernel(const uint2* __restrict__ cand, const uint32_t* __restric
 size_t topk_smem_bytes(int max_len) {
     const size_t words = (size_t)(max_len + 31) / 32;
     return sizeof(TopkScratch) + 2 * words * sizeof(uint32_t);
-}
-
-cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin,
-                        const int* row_len, int max_len, int k, int* idx, long long ld_idx,
-                        cudaStream_t stream, const DevCtx& ctx, const int* row_mask,
-                        int idx_offset) {
-    const size_t smem = topk_smem_bytes(max_len);
-    // fewer rows than SMs (a decode batch): one 1024-thread CTA per row shortens each
-    // row's chain of block-wide phases; otherwise two 512-thread CTAs per SM
-    const bool wide = rows < ctx.num_sms;
-    auto kernel = wide ? topk_radix_kernel<1024> : topk_radix_kernel<512>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    kernel<<<rows, wide ? 1024 : 512, smem, stream>>>(scores, ld, q_begin, row_len, max_len, k,
-                                                       idx, ld_idx, row_mask, idx_offset, ctx.err);
-    count_launch(DSA_KERNEL_TOPK);
-    return cudaGetLastError();
 }
 
 int topk_sample_max() { return kSampleMax; }

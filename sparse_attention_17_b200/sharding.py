@@ -64,3 +64,20 @@ def all_gather_rows(local, full, group=None) -> None:
         full.copy_(local)
         return
     dist.all_gather_into_tensor(full, local.contiguous(), group=group)
+
+
+def prefill_rank_rows(lib, q_idx, k_full, w, q, kv_full, blocks, k: int, scores, idx, out,
+                      scale: float) -> None:
+    """Step 3 for one rank: indexer + top-k per window of its query blocks into the index
+    buffer, then sparse MLA for those rows, through the library's C ABI (`lib` is the
+    sparse_attention_17_b200 module).  k_full / kv_full hold every token (after the
+    all-gather); q_idx, w, q, idx [T, k] and out [T, 16, 512] are indexed by token, and
+    only the rows of `blocks` are read or written; scores is a [window, ld] workspace."""
+    rw = scores.shape[0]
+    for q0, rows in blocks:
+        for w0 in range(q0, q0 + rows, rw):
+            wr = min(rw, q0 + rows - w0)
+            lib.indexer_scores(q_idx, k_full, w, scores, w0, wr)
+            lib.topk_select(scores, k, idx[w0:w0 + wr], q_begin=w0, rows=wr)
+        lib.sparse_mla_fwd(q[q0:q0 + rows], kv_full, idx[q0:q0 + rows], out[q0:q0 + rows],
+                           scale)

@@ -53,3 +53,30 @@ def test_reference_line_keys(monkeypatch):
     assert line["impl"] == "reference" and line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
     assert bench.run_reference(A, 1, 2) is None  # only rank 0 runs the oracle
+
+
+def test_tensor_peak_follows_the_clock_record():
+    """Burst peak when the timed region ran at the maximum SM clock without a power cap;
+    sustained otherwise (a kernel timed under the power cap)."""
+    peaks = {"bf16_tflops": 1646.6, "bf16_tflops_sustained": 1407.5}
+    at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped = {"sm_mhz": 1342.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    slow = {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.choose_tensor_peak(peaks, at_max)[0] == 1646.6
+    assert bench.choose_tensor_peak(peaks, capped)[0] == 1407.5
+    assert bench.choose_tensor_peak(peaks, slow)[0] == 1407.5
+    assert bench.choose_tensor_peak({"bf16_tflops": 1590.0}, capped)[0] == 1590.0
+    unsampled = {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+    assert bench.choose_tensor_peak(peaks, unsampled)[0] == 1407.5
+
+
+def test_reference_line_marks_extrapolated_step(monkeypatch):
+    from sparse_attention_17_b200 import inputs as G
+    monkeypatch.setattr(bench, "make_inputs", lambda T, k, seed, kv_dtype="bf16":
+                        G.mla_prefill_gauss(T=256, seed=seed, k=64))
+
+    class A:
+        T, topk, steps, warmup, cpu_seconds = 256, 64, 1, 0, 0.2
+
+    line = bench.run_reference(A, 0, 1)
+    assert line["extrapolated"] is True and line["sampled_ms_per_step"] > 0

@@ -127,19 +127,30 @@ def test_index_cache_stack_fss_x9():
     assert dsa.launch_count(0) == 9 * nwin
     assert dsa.launch_count(1) == 9 * nwin
     assert dsa.launch_count(2) == 27
-    # the buffer now holds the last F layer's (layer 24) indices: exact on sampled rows
+    # the buffer now holds the last F layer's (layer 24) indices: exact on every row
     rows = _sample_rows(T, k, seed=7, n_random=40)
     L24 = st["layers"][24]
     g_idx = idx.cpu().numpy()
-    for t in rows:
-        ref = O.prefill_indices(L24["q_idx"], L24["k_idx"], L24["w"], k, q_begin=int(t), rows=1)
-        check_indices_exact(g_idx[t:t + 1], ref, f"layer 24 row {t}")
-    # S layers 25, 26 reuse exactly those indices: bit-identical to a separate call
-    for l in (25, 26):
-        ref_out = torch.empty_like(outs[l])
-        dsa.sparse_mla_fwd(layers[l]["q"], layers[l]["kv"], idx, ref_out, G.SCALE_MLA)
-        torch.cuda.synchronize()
-        assert torch.equal(ref_out.view(torch.int16), outs[l].view(torch.int16)), l
+    check_indices_exact(g_idx, O.prefill_indices(L24["q_idx"], L24["k_idx"], L24["w"], k),
+                        "layer 24 indices, all rows")
+    # every F layer l: a separate dsa_indexer_scores + dsa_topk_select of its inputs, fed to
+    # separate attention calls of layers l, l+1, l+2, reproduces the stack's outputs bit
+    # for bit (the S layers used exactly the F layer's indices, and nothing else)
+    ld = (T + 3) // 4 * 4
+    sc = torch.empty((4096, ld), device="cuda")
+    for f in range(0, 27, 3):
+        idx_f = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        for q0 in range(0, T, 4096):
+            dsa.indexer_scores(layers[f]["q_idx"], layers[f]["k_idx"], layers[f]["w"], sc, q0,
+                               4096)
+            dsa.topk_select(sc, k, idx_f[q0:q0 + 4096], q_begin=q0, rows=4096)
+        for l in (f, f + 1, f + 2):
+            ref_out = torch.empty_like(outs[l])
+            dsa.sparse_mla_fwd(layers[l]["q"], layers[l]["kv"], idx_f, ref_out, G.SCALE_MLA)
+            torch.cuda.synchronize()
+            assert torch.equal(ref_out.view(torch.int16), outs[l].view(torch.int16)), l
+        if f == 24:
+            assert torch.equal(idx_f, idx)
     # sampled rows of F and S layers against the oracle (F layer 0 -> layers 0, 1, 2)
     L0 = st["layers"][0]
     ref_idx0 = np.stack([O.prefill_indices(L0["q_idx"], L0["k_idx"], L0["w"], k,

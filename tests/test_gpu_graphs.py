@@ -2,11 +2,14 @@
 full CUDA graphs): every call is asynchronous on the caller's stream, allocates nothing
 and never synchronises, so a captured sequence of calls must replay to bit-identical
 results -- also after new inputs are copied into the captured buffers."""
+import numpy as np
 import pytest
 import torch
 
 import sparse_attention_17_b200 as dsa
 from sparse_attention_17_b200 import inputs as G
+from oracle import oracle as O
+from parity import check_close_bf16, check_indices_exact
 
 pytestmark = pytest.mark.gpu
 
@@ -73,6 +76,16 @@ def test_layer_stack_graph_replay_bit_exact():
     assert torch.equal(idx, ref2_idx) and not torch.equal(ref2_idx, ref_idx)
     for a, b in zip(outs, ref2_outs):
         assert torch.equal(_bits(a), _bits(b))
+    # the replay against the oracle: the last F layer's indices on every row, and sampled
+    # rows of an F and an S layer computed from the oracle's indices
+    L6 = st2["layers"][6]
+    ref_i6 = O.prefill_indices(L6["q_idx"], L6["k_idx"], L6["w"], k)
+    check_indices_exact(idx, ref_i6, "graph replay: layer 6 indices")
+    rows = np.r_[0:8, 2040:2056, T - 8:T]
+    for l in (6, 8):
+        ref, _ = O.sparse_mla_prefill(st2["layers"][l]["q"][rows], st2["layers"][l]["kv"],
+                                      ref_i6[rows], G.SCALE_MLA)
+        check_close_bf16(outs[l][torch.from_numpy(rows).cuda()], ref, f"graph replay layer {l}")
 
 
 @pytest.mark.parametrize("fp8", [False, True])
@@ -109,3 +122,15 @@ def test_decode_step_graph_replay_bit_exact(fp8):
     torch.cuda.synchronize()
     assert torch.equal(idx, ref_idx)
     assert torch.equal(_bits(out), _bits(ref_out))
+    # the replay against the oracle: exact indices and the attention within the gate
+    o_sc = O.indexer_scores_decode(d["q_idx"], d["k_idx_pool"], d["w"], d["page_table"],
+                                   d["seq_lens"])
+    o_idx = O.topk(o_sc, d["seq_lens"].numpy(), k)
+    check_indices_exact(idx, o_idx, "decode graph replay indices")
+    if fp8:
+        o_out, o_lse = O.sparse_mla_fp8_decode(d["q"], d["kv_pool"], d["kv_scale"],
+                                               d["page_table"], o_idx, G.SCALE_MLA)
+    else:
+        o_out, o_lse = O.sparse_mla_decode(d["q"], d["kv_pool"], d["page_table"], o_idx,
+                                           G.SCALE_MLA)
+    check_close_bf16(out, o_out, "decode graph replay attention")

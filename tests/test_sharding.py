@@ -72,3 +72,54 @@ def test_all_gather_rows_two_gloo_ranks():
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
     assert res == {0: True, 1: True}
+
+
+def _oracle_rank_worker(rank, world, port, T, k, out):
+    """One rank of the row-sharded prefill with the CPU oracle as the compute: all-gather
+    the token shards of k_idx and the latent cache, then indices and attention for the
+    rank's zig-zag query blocks only."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from oracle import oracle as O
+        from sparse_attention_17_b200 import inputs as G
+        d = G.mla_prefill_int(T=T, k=k, seed=5)
+        s0, n = SH.token_shard(T, world, rank)
+        k_full = torch.empty_like(d["k_idx"])
+        kv_full = torch.empty_like(d["kv"])
+        SH.all_gather_rows(d["k_idx"][s0:s0 + n].contiguous(), k_full)
+        SH.all_gather_rows(d["kv"][s0:s0 + n].contiguous(), kv_full)
+        mine = []
+        for q0, rows in SH.zigzag_blocks(T, world, rank):
+            idx = O.prefill_indices(d["q_idx"], k_full, d["w"], k, q_begin=q0, rows=rows)
+            o, lse = O.sparse_mla_prefill(d["q"][q0:q0 + rows], kv_full, idx, G.SCALE_MLA)
+            mine.append((q0, rows, idx, o, lse))
+        allr = [None] * world
+        dist.all_gather_object(allr, mine)
+        if rank == 0:
+            out["blocks"] = [b for r in allr for b in r]
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("T,world", [(256, 2), (240, 3)])
+def test_row_sharded_oracle_prefill_equals_unsharded(T, world):
+    """Sharding is exact: ranks that all-gather the key and latent shards and compute only
+    their zig-zag blocks reproduce the unsharded indices and outputs bit for bit."""
+    from oracle import oracle as O
+    from sparse_attention_17_b200 import inputs as G
+    k = 64
+    port = _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        out = m.dict()
+        mp.spawn(_oracle_rank_worker, args=(world, port, T, k, out), nprocs=world, join=True)
+        blocks = out["blocks"]
+    d = G.mla_prefill_int(T=T, k=k, seed=5)
+    ref_idx = O.prefill_indices(d["q_idx"], d["k_idx"], d["w"], k)
+    ref_out, ref_lse = O.sparse_mla_prefill(d["q"], d["kv"], ref_idx, G.SCALE_MLA)
+    seen = torch.zeros(T, dtype=torch.int32)
+    for q0, rows, idx, o, lse in blocks:
+        seen[q0:q0 + rows] += 1
+        assert (idx == ref_idx[q0:q0 + rows]).all()
+        assert (o == ref_out[q0:q0 + rows]).all() and (lse == ref_lse[q0:q0 + rows]).all()
+    assert bool((seen == 1).all())
