@@ -12,12 +12,15 @@
 // consecutive TMEM columns that stay inside one thread -- no shuffles.
 //
 // Warp roles (640 threads): warp 0 issues TMA loads (query block once per unit, key tiles
-// through a ring of smem stages), warp 1 issues UMMAs into a double-buffered TMEM
-// accumulator (2 x 256 columns), warp 2 owns the TMEM allocation, warps 4..19 drain the
-// accumulator: tcgen05.ld, ReLU, weight, reduce, causal mask, coalesced fp32 stores.  The
+// through a ring of smem stages), warp 1 issues UMMAs into a ring of TMEM accumulators
+// (two of 256 columns in prefill), warp 2 owns the TMEM allocation, warps 4..19 drain the
+// accumulators: tcgen05.ld, ReLU, weight, reduce, causal mask, coalesced fp32 stores.  The
 // drain is the longest stage per tile (16 max + 16 multiply-adds per score), so it gets
-// four warps per TMEM lane quadrant, each on a quarter of the tile's queries, and the head
-// weights are applied with packed fp32x2 FMAs.
+// four warps per TMEM lane quadrant, each on a quarter of the block's queries, and the
+// weights are applied with packed fp32x2 FMAs (with at most two queries per warp their
+// head weights stay in registers for the whole unit; eight-query blocks, which allow
+// that, measured slower: less independent work per warp between the pipeline waits).  Tiles that lie wholly below the causal
+// diagonal of a full block store without a per-score test.
 //
 // Work units are (query block, chunk of at most 32 key tiles): prefill blocks hold 16
 // queries and their causal key range grows with the query position, so the range is cut
@@ -34,24 +37,29 @@ namespace {
 constexpr int kHI = 16;
 constexpr int kDI = 64;
 constexpr int kBM = 128;           // keys per tile (UMMA M)
-constexpr int kStages = 6;         // key-tile ring
+// Key-tile ring: 6 stages of 16 KB (a 12-stage ring for the one-query decode blocks
+// measured no faster).
+template <int QB>
+constexpr int stages_for() { return 6; }
 constexpr int kThreads = 640;
 constexpr int kEpiWarp0 = 4;       // first epilogue warp
 constexpr int kEpiWarps = 16;      // four per TMEM lane quadrant
 constexpr uint32_t kTileBytes = kBM * 128;  // 128 keys x 64 bf16
 constexpr int kDecodeChunkTiles = 16;       // decode unit = 2048 keys
 constexpr int kPrefillChunkTiles = 32;      // prefill unit: at most 4096 keys
+constexpr int kPrefillQB = 16;              // prefill queries per block (UMMA N = 256)
 static_assert(kPrefillChunkTiles * 128 == 4096, "filtered candidate lists are per 4096-key chunk");
 
 template <int QB>
 struct IdxSmem {
+    static constexpr int kStages = stages_for<QB>();
     alignas(1024) uint8_t k[kStages][kTileBytes];
     alignas(1024) uint8_t q[2][QB * kHI * 128 < 1024 ? 1024 : QB * kHI * 128];
     alignas(16) float w[2][QB * kHI];  // head weights of the unit's queries
     uint64_t k_full[kStages];
     uint64_t k_empty[kStages];
     uint64_t q_full[2], q_empty[2];
-    uint64_t acc_full[2], acc_empty[2];
+    uint64_t acc_full[4], acc_empty[4];
     uint32_t tmem_base;
     int abort;
     int pages[kDecodeChunkTiles * kBM / 16];  // decode: the unit's page-table entries
@@ -175,6 +183,7 @@ __device__ __forceinline__ bool produce_unit(IdxSmem<QB>& sm, const IdxParams& p
     tma_load_2d(sm.q[qb], tmap_q, 0, x.row0 * kHI, &sm.q_full[qb]);
     bulk_load(sm.w[qb], p.w + (long long)x.row0 * kHI, wbytes, &sm.q_full[qb]);
     for (int j = 0; j < x.ntiles; ++j, ++it) {
+        constexpr int kStages = IdxSmem<QB>::kStages;
         const int st = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
         if (!mbar_wait(&sm.k_empty[st], ph ^ 1, abort, p.err)) return false;
@@ -201,7 +210,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                   const __grid_constant__ CUtensorMap tmap_k, const IdxParams p) {
     constexpr int BN = QB * kHI;                     // UMMA N
     constexpr uint32_t kAccCols = BN < 32 ? 32 : BN;  // TMEM columns per accumulator
-    constexpr uint32_t kTmemCols = 2 * kAccCols <= 32 ? 32 : (2 * kAccCols <= 64 ? 64 : (2 * kAccCols <= 128 ? 128 : (2 * kAccCols <= 256 ? 256 : 512)));
+    // as many accumulators (at most 4) as the 512 TMEM columns hold: the MMA warp runs
+    // that many tiles ahead of the drain
+    constexpr int kAcc = 512 / kAccCols >= 4 ? 4 : (int)(512 / kAccCols);
+    constexpr uint32_t kTmemCols = kAcc * kAccCols <= 32 ? 32 : (kAcc * kAccCols <= 64 ? 64 : (kAcc * kAccCols <= 128 ? 128 : (kAcc * kAccCols <= 256 ? 256 : 512)));
     constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, 0, 0);
     using Smem = IdxSmem<QB>;
 
@@ -214,7 +226,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     volatile int* abort = &sm.abort;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) {
+        for (int i = 0; i < Smem::kStages; ++i) {
             mbar_init(&sm.k_full[i], 1);
             mbar_init(&sm.k_empty[i], 1);
         }
@@ -222,7 +234,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             mbar_init(&sm.q_full[i], 1);
             mbar_init(&sm.q_empty[i], 1 + kEpiWarps);  // UMMA commit + epilogue warps
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kAcc; ++i) {
             mbar_init(&sm.acc_full[i], 1);
             mbar_init(&sm.acc_empty[i], kEpiWarps);
         }
@@ -284,10 +296,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const uint32_t q_addr = smem_u32(sm.q[qb]);
             bool ok = true;
             for (int j = 0; j < x.ntiles; ++j, ++it) {
-                const int st = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
-                const int ab = it & 1;
-                const uint32_t aph = (it >> 1) & 1;
+                const int st = it % Smem::kStages;
+                const uint32_t ph = (it / Smem::kStages) & 1;
+                const int ab = it % kAcc;
+                const uint32_t aph = (it / kAcc) & 1;
                 if (!mbar_wait(&sm.k_full[st], ph, abort, p.err)) { ok = false; break; }
                 if (!mbar_wait(&sm.acc_empty[ab], aph ^ 1, abort, p.err)) { ok = false; break; }
                 tc_fence_after();
@@ -308,6 +320,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         const int quad = warp & 3;              // TMEM lane quadrant this warp may access
         const int part = ew >> 2;               // which quarter of the queries
         constexpr int QPW = QB >= 4 ? QB / 4 : 1;  // queries per epilogue warp
+        // with at most two queries per warp their 32 head weights stay in registers for
+        // the whole unit; otherwise they are read from shared memory per tile
+        constexpr bool kHoist = QPW <= 2;
         const bool active = QB >= 4 || part == 0;
         uint32_t it = 0;
         for (int i = 0, ui = 0;; ++i, ++ui) {
@@ -317,6 +332,17 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const int qb = ui & 1;
             if (!mbar_wait(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err)) break;
             const float* wbuf = sm.w[qb] + part * QPW * kHI;  // this warp's queries' weights
+            float wreg[kHoist ? QPW * kHI : 1];
+            if constexpr (kHoist) {
+#pragma unroll
+                for (int h4 = 0; h4 < QPW * kHI / 4; ++h4) {
+                    const float4 wv = reinterpret_cast<const float4*>(wbuf)[h4];
+                    wreg[4 * h4] = wv.x;
+                    wreg[4 * h4 + 1] = wv.y;
+                    wreg[4 * h4 + 2] = wv.z;
+                    wreg[4 * h4 + 3] = wv.w;
+                }
+            }
             float tau[QPW];      // kFilter: the thresholds of this warp's queries as floats
             uint32_t ncand[QPW]; // kFilter: candidates this warp appended per query
 #pragma unroll
@@ -331,12 +357,15 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const int chunk = x.tile0 / kPrefillChunkTiles;
             bool ok = true;
             for (int j = 0; j < x.ntiles; ++j, ++it) {
-                const int ab = it & 1;
-                const uint32_t aph = (it >> 1) & 1;
+                const int ab = it % kAcc;
+                const uint32_t aph = (it / kAcc) & 1;
                 if (!mbar_wait(&sm.acc_full[ab], aph, abort, p.err)) { ok = false; break; }
                 tc_fence_after();
                 const int lt = x.tile0 + j;  // logical tile
-                const int s = lt * (PAGED ? 1 : p.tile_stride) * kBM + quad * 32 + lane;
+                const int tile_key0 = lt * (PAGED ? 1 : p.tile_stride) * kBM;
+                const int s = tile_key0 + quad * 32 + lane;
+                // every key of the tile precedes every query of the block: no causal test
+                const bool below = !PAGED && tile_key0 + kBM - 1 <= x.row0 && x.len == QB;
                 const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + ab * kAccCols;
                 if (active) {
                     constexpr int QW = QPW < 2 ? QPW : 2;  // queries per TMEM load round
@@ -350,13 +379,18 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
                         for (int qq = 0; qq < QW; ++qq) {
                             const int qidx = i0 + qq;
-                            const float4* w4 =
-                                reinterpret_cast<const float4*>(wbuf + (qidx - part * QPW) * kHI);
+                            const int qo = qidx - part * QPW;
                             // even heads accumulate in acc0, odd heads in acc1
                             float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
                             for (int h4 = 0; h4 < 4; ++h4) {
-                                const float4 wv = w4[h4];
+                                float4 wv;
+                                if constexpr (kHoist) {
+                                    wv = make_float4(wreg[qo * kHI + 4 * h4], wreg[qo * kHI + 4 * h4 + 1],
+                                                     wreg[qo * kHI + 4 * h4 + 2], wreg[qo * kHI + 4 * h4 + 3]);
+                                } else {
+                                    wv = reinterpret_cast<const float4*>(wbuf + qo * kHI)[h4];
+                                }
                                 const uint32_t* rv = r[qq] + 4 * h4;
                                 ffma2(acc0, acc1, wv.x, wv.y, fmaxf(__uint_as_float(rv[0]), 0.f),
                                       fmaxf(__uint_as_float(rv[1]), 0.f));
@@ -368,7 +402,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                                 if (s < x.len) p.scores[(long long)x.row0 * p.ld + s] = score;
                             } else if constexpr (MODE == kDense) {
                                 const int t = x.row0 + qidx;
-                                if (qidx < x.len && s <= t)
+                                if (below || (qidx < x.len && s <= t))
                                     p.scores[(long long)(t - p.q_begin) * p.ld + s] = score;
                             } else if constexpr (MODE == kSample) {
                                 // compact sample row: logical tile lt at columns lt*128..
@@ -382,7 +416,6 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                                 const int t = x.row0 + qidx;
                                 const long long r = t - p.q_begin;
                                 const bool valid = qidx < x.len && s <= t;
-                                const int qo = qidx - part * QPW;
                                 const bool gt = valid && score >= tau[qo];
                                 const unsigned gtm = __ballot_sync(0xffffffffu, gt);
                                 if (gtm) {
@@ -444,7 +477,7 @@ cudaError_t launch_indexer_tc(const CUtensorMap& tq, const CUtensorMap& tk, cons
 template <int MODE>
 cudaError_t launch_prefill(const __nv_bfloat16* q_idx, const __nv_bfloat16* k_idx, int T, int S,
                            IdxParams p, cudaStream_t stream, const DevCtx& ctx) {
-    constexpr int QB = 16;
+    constexpr int QB = kPrefillQB;
     CUtensorMap tq, tk;
     if (!make_tmap_bf16_2d(&tq, q_idx, (uint64_t)T * kHI, kDI, kDI * 2, QB * kHI, kDI))
         return cudaErrorInvalidValue;

@@ -51,8 +51,7 @@ struct SCfg {
 };
 
 struct StreamSmem {
-    uint32_t key[kCap];           // candidate scores (float bits)
-    uint8_t off[kCap];            // candidate position within its chunk
+    uint2 cand[kCap];             // candidates: {score bits, position within the chunk}
     uint32_t hist[2][256];        // radix histograms, alternating between rounds
     uint32_t red[32][2];          // per-warp partials of a reduction
     uint32_t scan[32];
@@ -60,12 +59,6 @@ struct StreamSmem {
     uint32_t bcast[2];
     // followed by chunk_start[nchunk] (uint16) and chunk_cnt[nchunk] (uint8)
 };
-
-__device__ __forceinline__ uint32_t lanemask_lt() {
-    uint32_t m;
-    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-    return m;
-}
 
 // The float threshold equivalent to an order key: float_order_key(x) >= key0 exactly when
 // x >= key_to_float_lower(key0), for key0 != 0 and x not NaN.
@@ -346,7 +339,6 @@ topk_stream_kernel(const float* __restrict__ scores, long long ld, int rows, int
     // ---- stream: every key >= tau0 to the candidate buffer, chunk by chunk ----
     const int nch = (n + kChunk - 1) / kChunk;
     const int nfull = n / kChunk;  // chunks that lie entirely inside the row
-    const uint32_t lt = lanemask_lt();
     for (int c0 = warp; c0 < nch; c0 += C::kWarps * C::kUnroll) {
         float4 v[C::kUnroll];
 #pragma unroll
@@ -362,43 +354,53 @@ topk_stream_kernel(const float* __restrict__ scores, long long ld, int rows, int
                 v[u].w = s0 + 3 < n ? __ldcs(row + s0 + 3) : __int_as_float(0x7fc00000);
             }
         }
-        unsigned bal[C::kUnroll][4];
-        uint32_t cnt[C::kUnroll], tot = 0;
+        // per lane: the 4-bit take mask of each unrolled chunk, and the counts packed one
+        // byte per chunk (at most 4 per lane, 128 per chunk: no byte overflows), so that
+        // one warp scan places the candidates of all of them
+        uint32_t msk[C::kUnroll], packed = 0;
 #pragma unroll
         for (int u = 0; u < C::kUnroll; ++u) {
-            bal[u][0] = __ballot_sync(0xffffffffu, v[u].x >= tau0f);
-            bal[u][1] = __ballot_sync(0xffffffffu, v[u].y >= tau0f);
-            bal[u][2] = __ballot_sync(0xffffffffu, v[u].z >= tau0f);
-            bal[u][3] = __ballot_sync(0xffffffffu, v[u].w >= tau0f);
-            cnt[u] = __popc(bal[u][0]) + __popc(bal[u][1]) + __popc(bal[u][2]) + __popc(bal[u][3]);
-            tot += cnt[u];
+            msk[u] = (v[u].x >= tau0f ? 1u : 0u) | (v[u].y >= tau0f ? 2u : 0u) |
+                     (v[u].z >= tau0f ? 4u : 0u) | (v[u].w >= tau0f ? 8u : 0u);
+            packed |= (uint32_t)__popc(msk[u]) << (8 * u);
         }
+        uint32_t incl = packed;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t chunk_tot = __shfl_sync(0xffffffffu, incl, 31);  // per-chunk totals
+        const uint32_t excl = incl - packed;
+        uint32_t tot = 0;
+#pragma unroll
+        for (int u = 0; u < C::kUnroll; ++u) tot += (chunk_tot >> (8 * u)) & 0xFFu;
         uint32_t base = 0;
         if (lane == 0 && tot) base = atomicAdd(&sm.ncand, tot);
         base = __shfl_sync(0xffffffffu, base, 0);
 #pragma unroll
         for (int u = 0; u < C::kUnroll; ++u) {
             const int c = c0 + u * C::kWarps;
+            const uint32_t cnt = (chunk_tot >> (8 * u)) & 0xFFu;
             if (c < nch) {
                 if (lane == 0) {
                     chunk_start[c] = (uint16_t)min(base, 0xFFFFu);
-                    chunk_cnt[c] = (uint8_t)cnt[u];
+                    chunk_cnt[c] = (uint8_t)cnt;
                 }
-                uint32_t pos = base + __popc(bal[u][0] & lt) + __popc(bal[u][1] & lt) +
-                               __popc(bal[u][2] & lt) + __popc(bal[u][3] & lt);
-                const float xv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                // a chunk past the buffer's end sends the row to the exact path
+                if (base + cnt <= (uint32_t)kCap) {
+                    uint32_t pos = base + ((excl >> (8 * u)) & 0xFFu);
+                    const float xv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    if ((bal[u][e] >> lane) & 1u) {
-                        if (pos < (uint32_t)kCap) {
-                            sm.key[pos] = __float_as_uint(xv[e]);
-                            sm.off[pos] = (uint8_t)(4 * lane + e);
+                    for (int e = 0; e < 4; ++e) {
+                        if ((msk[u] >> e) & 1u) {
+                            sm.cand[pos] = make_uint2(__float_as_uint(xv[e]), (uint32_t)(4 * lane + e));
+                            ++pos;
                         }
-                        ++pos;
                     }
                 }
             }
-            base += cnt[u];
+            base += cnt;
         }
     }
     __syncthreads();
@@ -413,7 +415,7 @@ topk_stream_kernel(const float* __restrict__ scores, long long ld, int rows, int
 #pragma unroll
     for (int i = 0; i < C::kCPT; ++i) {
         const uint32_t j = threadIdx.x + i * NT;
-        ck[i] = j < ncand ? float_order_key(__uint_as_float(sm.key[j])) : 0u;
+        ck[i] = j < ncand ? float_order_key(__uint_as_float(sm.cand[j].x)) : 0u;
     }
     uint32_t mn, mx, need;
     block_minmax<NT, C::kCPT>(ck, &mn, &mx, sm);
@@ -430,7 +432,7 @@ topk_stream_kernel(const float* __restrict__ scores, long long ld, int rows, int
     for (int c = ca; c < cb; ++c) {
         const int st = chunk_start[c], ct = chunk_cnt[c];
         for (int j = st; j < st + ct; ++j) {
-            const uint32_t key = float_order_key(__uint_as_float(sm.key[j]));
+            const uint32_t key = float_order_key(__uint_as_float(sm.cand[j].x));
             packed += key > tau ? 1u : (key == tau ? 0x10000u : 0u);
         }
     }
@@ -440,8 +442,9 @@ topk_stream_kernel(const float* __restrict__ scores, long long ld, int rows, int
     for (int c = ca; c < cb; ++c) {
         const int st = chunk_start[c], ct = chunk_cnt[c];
         for (int j = st; j < st + ct; ++j) {
-            const uint32_t key = float_order_key(__uint_as_float(sm.key[j]));
-            const int s = c * kChunk + sm.off[j] + idx_offset;
+            const uint2 cj = sm.cand[j];
+            const uint32_t key = float_order_key(__uint_as_float(cj.x));
+            const int s = c * kChunk + (int)cj.y + idx_offset;
             if (key > tau) {
                 out[sb + min(tb, need)] = s;
                 ++sb;
@@ -479,3 +482,4 @@ cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin
 }
 
 }  // namespace dsa
+
