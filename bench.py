@@ -39,6 +39,12 @@ def parse_args(argv=None):
     ap.add_argument("--topk", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode workload that the default prefill line carries as "
+                         "its nested 'decode' object")
+    ap.add_argument("--no-rows", action="store_true",
+                    help="N>1: skip the row-sharded strong-scaling measurement that the "
+                         "default line carries as its nested 'strong_scaling' object")
     ap.add_argument("--workload", choices=["prefill", "decode", "stack", "varlen"],
                     default="prefill",
                     help="prefill: the T=65536 headline; decode: 64 sequences x 32768 paged "
@@ -675,6 +681,11 @@ def run_decode(args, local_rank):
     peaks, src = load_peaks()
     gather = B * k * (576 if fp8 else 1152)
     kidx = B * L * 64 * 2
+    # algorithmic HBM bytes of a step: indexer keys, the dense score row written and read
+    # once, the gathered latent rows, queries, indices and outputs
+    step_bytes = (kidx + 2 * B * L * 4 + gather + B * 16 * 576 * 2 + B * (16 * 64 * 2 + 16 * 4)
+                  + B * k * 4 * 2 + B * 16 * 512 * 2)
+    step_roof_ms = step_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3
     return {"metric": "DSA decode sequences/sec (64 x 32768 paged, top-2048)", "value":
             round(B / (ms / 1e3), 1), "unit": "sequences/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
@@ -689,6 +700,11 @@ def run_decode(args, local_rank):
                         "mla_gather_gbs": round(gather / (t_mla / 1e3) / 1e9, 1),
                         "mla_gather_frac_of_hbm": round(gather / (t_mla / 1e3) / 1e9
                                                         / peaks["hbm_gbs"], 4),
+                        "indexer_key_read_frac_of_hbm": round(kidx / (t_idx / 1e3) / 1e9
+                                                              / peaks["hbm_gbs"], 4),
+                        "step_hbm_bytes": step_bytes,
+                        "step_hbm_roofline_ms": round(step_roof_ms, 4),
+                        "step_frac_of_hbm_roofline": round(step_roof_ms / ms, 4),
                         "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": src}}
 
 
@@ -832,6 +848,21 @@ def main(argv=None):
             res = run_rows(args, rank, world, local_rank)
         else:
             res = run_native(args, rank, world, local_rank)
+            if world > 1 and not args.no_rows:
+                # the same prefill split over the ranks by query rows (every rank takes part)
+                rows_line = run_rows(args, rank, world, local_rank)
+                if res is not None:
+                    res["strong_scaling"] = {kk: rows_line[kk] for kk in
+                                             ("value", "unit", "ms_per_step", "scaling", "config")}
+            if world == 1 and res is not None and not args.no_decode:
+                # the batched decode workload, measured in the same run (a nested object,
+                # so that the line stays one line)
+                import torch
+                torch.cuda.synchronize()
+                dec = run_decode(args, local_rank)
+                res["decode"] = {kk: dec[kk] for kk in ("metric", "value", "unit", "ms_per_step",
+                                                       "kernels", "cuda_graph", "derived",
+                                                       "config")}
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -216,6 +216,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     constexpr uint32_t kTmemCols = kAcc * kAccCols <= 32 ? 32 : (kAcc * kAccCols <= 64 ? 64 : (kAcc * kAccCols <= 128 ? 128 : (kAcc * kAccCols <= 256 ? 256 : 512)));
     constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, 0, 0);
     using Smem = IdxSmem<QB>;
+    // One query per block (decode): the four query quarters of the epilogue take turns on
+    // the tiles, each with an accumulator of its own, so four tiles drain at a time
+    // instead of one tile by a quarter of the warps.
+    constexpr bool kSplitTiles = QB == 1;
+    static_assert(!kSplitTiles || kAcc == 4, "tile turns need one accumulator per quarter");
 
     static_assert(MODE == kDense || !PAGED, "decode stores dense rows");
     if (p.guard != nullptr && *p.guard == 0) return;  // a fallback launch with nothing to do
@@ -236,7 +241,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         }
         for (int i = 0; i < kAcc; ++i) {
             mbar_init(&sm.acc_full[i], 1);
-            mbar_init(&sm.acc_empty[i], kEpiWarps);
+            mbar_init(&sm.acc_empty[i], kSplitTiles ? 4 : kEpiWarps);
         }
         sm.abort = 0;
         fence_barrier_init();
@@ -252,13 +257,32 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
-        // Lane 0 issues the copies.  For paged keys the whole warp first reads the unit's
-        // page-table entries into shared memory: one round trip per unit instead of a
-        // dependent load before every tile's copies.
+        // Lane 0 issues the copies.  For paged keys the whole warp reads a unit's page-table
+        // entries into shared memory first (one round trip per unit, not a dependent load
+        // before every tile's copies), and the next unit's entries are loaded into
+        // registers while lane 0 issues this unit's copies, so that round trip overlaps them.
         if (lane == 0) {
             tma_prefetch_desc(&tmap_q);
             tma_prefetch_desc(&tmap_k);
         }
+        constexpr int kPgLane = kDecodeChunkTiles * kBM / 16 / 32;  // entries per lane (pages >= 16)
+        int pg_next[kPgLane];
+        auto load_pages = [&](int u, int (&dst)[kPgLane]) {
+            if constexpr (PAGED) {
+                if (u < p.num_units) {
+                    const UnitInfo<QB, PAGED> y = unit_info<QB, PAGED>(p, u);
+                    const int per = kBM / p.page_size;
+                    const int npg = min(y.ntiles * per, (y.len - y.tile0 * kBM + p.page_size - 1) / p.page_size);
+                    const int* pt = p.page_table + (long long)y.row0 * p.max_pages + y.tile0 * per;
+#pragma unroll
+                    for (int i = 0; i < kPgLane; ++i) {
+                        const int q = lane + 32 * i;
+                        dst[i] = q < npg ? __ldg(pt + q) : 0;
+                    }
+                }
+            }
+        };
+        load_pages(unit_at(0), pg_next);
         uint32_t it = 0;
         for (int i = 0, ui = 0;; ++i, ++ui) {
             const int u = unit_at(i);
@@ -267,16 +291,20 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             if constexpr (PAGED) {
                 const int per = kBM / p.page_size;
                 const int npg = min(x.ntiles * per, (x.len - x.tile0 * kBM + p.page_size - 1) / p.page_size);
-                const int* pt = p.page_table + (long long)x.row0 * p.max_pages + x.tile0 * per;
-                for (int q = lane; q < npg; q += 32) {
-                    int pg = __ldg(pt + q);
-                    if (pg < 0 || pg >= p.num_pages) {
-                        atomicOr(p.err, DSA_DEVERR_PAGE_RANGE);
-                        pg = 0;
+#pragma unroll
+                for (int j = 0; j < kPgLane; ++j) {
+                    const int q = lane + 32 * j;
+                    if (q < npg) {
+                        int pg = pg_next[j];
+                        if (pg < 0 || pg >= p.num_pages) {
+                            atomicOr(p.err, DSA_DEVERR_PAGE_RANGE);
+                            pg = 0;
+                        }
+                        sm.pages[q] = pg;
                     }
-                    sm.pages[q] = pg;
                 }
                 __syncwarp();
+                load_pages(unit_at(i + 1), pg_next);
             }
             bool ok = true;
             if (lane == 0) ok = produce_unit<QB, PAGED>(sm, p, x, ui, it, &tmap_q, &tmap_k, abort);
@@ -323,7 +351,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
         // with at most two queries per warp their 32 head weights stay in registers for
         // the whole unit; otherwise they are read from shared memory per tile
         constexpr bool kHoist = QPW <= 2;
-        const bool active = QB >= 4 || part == 0;
+        const bool active = QB >= 4 || kSplitTiles;
+        const int qbase = kSplitTiles ? 0 : part * QPW;  // this warp's first query of the block
         uint32_t it = 0;
         for (int i = 0, ui = 0;; ++i, ++ui) {
             const int u = unit_at(i);
@@ -331,7 +360,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             const UnitInfo<QB, PAGED> x = unit_info<QB, PAGED>(p, u);
             const int qb = ui & 1;
             if (!mbar_wait(&sm.q_full[qb], (ui >> 1) & 1, abort, p.err)) break;
-            const float* wbuf = sm.w[qb] + part * QPW * kHI;  // this warp's queries' weights
+            const float* wbuf = sm.w[qb] + qbase * kHI;  // this warp's queries' weights
             float wreg[kHoist ? QPW * kHI : 1];
             if constexpr (kHoist) {
 #pragma unroll
@@ -347,10 +376,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             uint32_t ncand[QPW]; // kFilter: candidates this warp appended per query
 #pragma unroll
             for (int qi = 0; qi < QPW; ++qi) {
-                const int r = x.row0 + part * QPW + qi - p.q_begin;
+                const int r = x.row0 + qbase + qi - p.q_begin;
                 // an order key >= tau[r] is exactly a score >= the float the key stands for
                 const uint32_t tk =
-                    (MODE == kFilter && part * QPW + qi < x.len) ? __ldg(p.tau + r) : 0u;
+                    (MODE == kFilter && qbase + qi < x.len) ? __ldg(p.tau + r) : 0u;
                 tau[qi] = __uint_as_float((tk & 0x80000000u) ? (tk & 0x7FFFFFFFu) : ~tk);
                 ncand[qi] = 0u;
             }
@@ -359,6 +388,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             for (int j = 0; j < x.ntiles; ++j, ++it) {
                 const int ab = it % kAcc;
                 const uint32_t aph = (it / kAcc) & 1;
+                if (kSplitTiles && ab != part) continue;  // another quarter drains this tile
                 if (!mbar_wait(&sm.acc_full[ab], aph, abort, p.err)) { ok = false; break; }
                 tc_fence_after();
                 const int lt = x.tile0 + j;  // logical tile
@@ -372,14 +402,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
 #pragma unroll
                     for (int qi = 0; qi < QPW; qi += QW) {
                         uint32_t r[QW][16];
-                        const int i0 = part * QPW + qi;
+                        const int i0 = qbase + qi;
 #pragma unroll
                         for (int qq = 0; qq < QW; ++qq) tmem_ld16(tbase + (i0 + qq) * kHI, r[qq]);
                         tmem_wait_ld();
 #pragma unroll
                         for (int qq = 0; qq < QW; ++qq) {
                             const int qidx = i0 + qq;
-                            const int qo = qidx - part * QPW;
+                            const int qo = qidx - qbase;
                             // even heads accumulate in acc0, odd heads in acc1
                             float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
@@ -435,11 +465,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
             }
             if (!ok) break;
             if constexpr (MODE == kFilter) {
-                if (active && lane < QPW && part * QPW + lane < x.len) {
+                if (active && lane < QPW && qbase + lane < x.len) {
                     uint32_t nc = 0;
 #pragma unroll
                     for (int qi = 0; qi < QPW; ++qi) nc = lane == qi ? ncand[qi] : nc;
-                    const long long r = x.row0 + part * QPW + lane - p.q_begin;
+                    const long long r = x.row0 + qbase + lane - p.q_begin;
                     p.ccount[(r * p.nchunk_max + chunk) * 4 + quad] = nc;
                 }
             }
