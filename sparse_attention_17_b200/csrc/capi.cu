@@ -495,8 +495,8 @@ size_t dsa_layer_stack_workspace_size(int T, int rows_window) {
     if (rw <= 0) {
         // default: about 4 GB of scores per window.  Wider windows give the indexer and
         // top-k launches more rows per launch and fewer launch tails: at T = 65536 this is
-        // 16384 rows, and the index phase measured 13.9 / 13.2 / 12.8 / 12.5 / 12.4 ms with
-        // 2048 / 4096 / 8192 / 16384 / 32768-row windows.
+        // 16384 rows, and the index phase measured 10.42 / 10.12 / 9.83 / 9.76 ms with
+        // 4096 / 8192 / 16384 / 32768-row windows.
         rw = (4096ll << 20) / (ld * 4);
         if (rw < 128) rw = 128;
     }
