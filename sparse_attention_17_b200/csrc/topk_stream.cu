@@ -6,8 +6,9 @@
 // n <= k every key is selected.  Output: the selected key positions in ascending order,
 // then -1 padding.
 //
-// One small CTA per row (256 threads, about 22 KB of shared memory, so several rows are
-// in flight on every SM; 1024 threads when a launch has fewer rows than the GPU has SMs).
+// One small CTA per row (256 threads, about 36 KB of shared memory at 65536 keys, so four
+// rows are in flight on every SM; 1024 threads when a launch has fewer rows than the GPU
+// has SMs), longest rows first.
 // Scores map to order-preserving uint32 keys (-0 like +0).
 //   sample  rows longer than the candidate buffer load up to 4096 scores (32-key pieces
 //           spread evenly over the row) into registers; radix selection (8-bit digits,
@@ -15,11 +16,13 @@
 //           16 bits of the sample key of rank e + 4 sqrt(e) + 2, e = the number of samples
 //           expected above the row's k-th largest score; the lower edge tau0 of that
 //           16-bit bin is the provisional threshold;
-//   stream  one pass over the row, 128-key chunks (one 16-byte load per lane) dealt to the
-//           warps round-robin: every score >= tau0 goes to the candidate buffer, the
-//           chunk's candidates contiguous and in index order at a place reserved with one
-//           shared atomic per warp and unrolled group of chunks; each chunk records where
-//           its candidates start and how many there are;
+//   stream  one pass over the row, 128-key chunks (one 16-byte load per lane), four per
+//           warp and iteration, dealt to the warps round-robin: every score >= tau0 goes to
+//           the candidate buffer as {score bits, position in the chunk}, the chunk's candidates
+//           contiguous and in index order.  Each lane's 4-bit take mask per chunk and the
+//           counts packed one byte per chunk give, after one warp scan, every candidate its
+//           place in a range reserved with one shared atomic per warp and iteration; each
+//           chunk records where its candidates start and how many there are;
 //   select  the candidates' keys move to registers; radix selection with 8-bit digits
 //           (a shared histogram per digit, two barriers) below the bits that the smallest
 //           and largest candidate share gives the k-th largest key tau and `need`, the
