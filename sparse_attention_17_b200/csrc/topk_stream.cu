@@ -69,6 +69,13 @@ __device__ __forceinline__ float order_key_to_float(uint32_t key0) {
     return __uint_as_float((key0 & 0x80000000u) ? (key0 & 0x7FFFFFFFu) : ~key0);
 }
 
+// Bits pos .. pos + len - 1 of v (PTX bfe: one instruction).
+__device__ __forceinline__ uint32_t bfe_u32(uint32_t v, int pos, int len) {
+    uint32_t r;
+    asm("bfe.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(v), "r"(pos), "r"(len));
+    return r;
+}
+
 // Block-wide minimum and maximum of the keys that are not 0 (0 marks an absent entry).
 template <int NT, int N>
 __device__ __forceinline__ void block_minmax(const uint32_t (&keys)[N], uint32_t* mn_out,
@@ -141,11 +148,19 @@ __device__ uint32_t block_radix_select(const uint32_t (&keys)[N], uint32_t rank,
         uint32_t* hist = sm.hist[h];
         for (int i = threadIdx.x; i < 256; i += NT) sm.hist[h ^ 1][i] = 0u;
         const uint32_t hp = b >= 32 ? 0u : prefix >> b;
-        const uint32_t dmask = (1u << d) - 1u;
+        if (b < 32 && hp != 0u) {
+            // an absent entry (key 0) cannot match a non-zero prefix: no test for it
 #pragma unroll
-        for (int i = 0; i < N; ++i) {
-            const uint32_t key = keys[i];
-            if (key != 0u && (b >= 32 || (key >> b) == hp)) atomicAdd(&hist[(key >> s) & dmask], 1u);
+            for (int i = 0; i < N; ++i) {
+                const uint32_t key = keys[i];
+                if ((key >> b) == hp) atomicAdd(&hist[bfe_u32(key, s, d)], 1u);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const uint32_t key = keys[i];
+                if (key != 0u && (b >= 32 || (key >> b) == hp)) atomicAdd(&hist[bfe_u32(key, s, d)], 1u);
+            }
         }
         __syncthreads();
         if (warp == 0) find_digit_from_top(hist, rank, sm);
@@ -429,14 +444,17 @@ topk_stream_kernel(const float* __restrict__ scores, long long ld, int rows, int
     const uint32_t tau = block_radix_select<NT, C::kCPT>(ck, (uint32_t)k, fixed, hi, 0, sm, &need);
 
     // ---- output: threads take consecutive chunks; one scan places every selected key ----
+    // (scores are compared as floats with tau's own value: x > tauf exactly when
+    // float_order_key(x) > tau, and x == tauf when the keys are equal, -0 == +0 included)
+    const float tauf = order_key_to_float(tau);
     const int cpt = (nch + NT - 1) / NT;
     const int ca = min((int)threadIdx.x * cpt, nch), cb = min(ca + cpt, nch);
     uint32_t packed = 0;
     for (int c = ca; c < cb; ++c) {
         const int st = chunk_start[c], ct = chunk_cnt[c];
         for (int j = st; j < st + ct; ++j) {
-            const uint32_t key = float_order_key(__uint_as_float(sm.cand[j].x));
-            packed += key > tau ? 1u : (key == tau ? 0x10000u : 0u);
+            const float x = __uint_as_float(sm.cand[j].x);
+            packed += x > tauf ? 1u : (x == tauf ? 0x10000u : 0u);
         }
     }
     uint32_t total;
@@ -446,12 +464,12 @@ topk_stream_kernel(const float* __restrict__ scores, long long ld, int rows, int
         const int st = chunk_start[c], ct = chunk_cnt[c];
         for (int j = st; j < st + ct; ++j) {
             const uint2 cj = sm.cand[j];
-            const uint32_t key = float_order_key(__uint_as_float(cj.x));
+            const float x = __uint_as_float(cj.x);
             const int s = c * kChunk + (int)cj.y + idx_offset;
-            if (key > tau) {
+            if (x > tauf) {
                 out[sb + min(tb, need)] = s;
                 ++sb;
-            } else if (key == tau) {
+            } else if (x == tauf) {
                 if (tb < need) out[sb + tb] = s;
                 ++tb;
             }
