@@ -275,6 +275,31 @@ def test_topk_one_warp_region_overflows_to_exact():
     check_indices_exact(idx, ref, "one-warp overflow")
 
 
+@pytest.mark.parametrize("rows,S,vals", [(5, 70000, 40), (40, 9000, 3), (60, 4200, 1000),
+                                         (2, 5000, 2), (74, 20000, 5), (100, 20000, 1000),
+                                         (147, 2600, 7)])
+def test_topk_few_rows_split_over_a_cluster(rows, S, vals):
+    """Launches with at most half as many rows as SMs split each row's candidate pass over
+    a cluster of two CTAs (ranges of chunks that need not fill a whole pass of the CTA's
+    warps) and gather the candidates in the first; up to one row per SM, one 1024-thread
+    CTA per row.  Row lengths spread over [k+1, S], ties within and across the CTAs'
+    ranges, and one causal window of the same number of rows."""
+    r = np.random.default_rng(rows * 7 + S)
+    k = 2048
+    sc = r.integers(0, vals, (rows, S)).astype(np.float64)
+    n_valid = list(r.integers(k + 1, S + 1, rows))
+    n_valid[0] = S
+    idx, ref = _topk_case(sc, n_valid, k, row_len=True)
+    check_indices_exact(idx, ref, f"{rows} rows of up to {S} keys")
+    q_begin = S - rows
+    ld = (S + 3) // 4 * 4
+    buf = torch.zeros((rows, ld))
+    buf[:, :S] = torch.from_numpy(sc)
+    idx = torch.empty((rows, k), dtype=torch.int32, device="cuda")
+    dsa.topk_select(buf.cuda(), k, idx, q_begin=q_begin, rows=rows)
+    check_indices_exact(idx, O.topk(sc, O.causal_n_valid(q_begin, rows), k), "causal window")
+
+
 @pytest.mark.parametrize("n_valid", [[3072, 3073, 3071, 8192, 8193, 12345, 2049, 65536, 16385,
                                       4097, 3840, 3841]])
 def test_topk_lengths_around_sample_switch(n_valid):
