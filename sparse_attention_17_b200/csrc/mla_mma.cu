@@ -612,10 +612,16 @@ sparse_mla_mma_kernel(const Params p) {
 }
 
 // Merge of decode splits: lse = log sum_i exp(lse_i); out = sum_i exp(lse_i - lse) o_i.
-__global__ void mla_combine_kernel(const float* __restrict__ o_part,
-                                   const float* __restrict__ lse_part, int splits,
-                                   __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+// Grid (sequences, kCombineParts): each CTA merges one part of the output dims for all 16
+// heads (a warp per head), so that a decode batch spreads over the SMs and every lane has
+// kDv / 32 / kCombineParts independent loads per split in flight.
+constexpr int kCombineParts = 4;
+constexpr int kCombineDims = kDv / kCombineParts;
+__global__ void __launch_bounds__(kH * 32)
+mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                   int splits, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     const int n = blockIdx.x;
+    const int d0 = blockIdx.y * kCombineDims;
     const int h = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const float* lp = lse_part + (long long)n * splits * kH;
@@ -626,21 +632,22 @@ __global__ void mla_combine_kernel(const float* __restrict__ o_part,
         const float l = lp[i * kH + h];
         denom += l == -INFINITY ? 0.f : expf(l - mx);
     }
-    float acc[kDv / 32];
+    float acc[kCombineDims / 32];
 #pragma unroll
-    for (int d = 0; d < kDv / 32; ++d) acc[d] = 0.f;
+    for (int d = 0; d < kCombineDims / 32; ++d) acc[d] = 0.f;
+#pragma unroll 4
     for (int i = 0; i < splits; ++i) {
         const float l = lp[i * kH + h];
         if (l == -INFINITY) continue;
         const float wgt = expf(l - mx) / denom;
-        const float* op = o_part + (((long long)n * splits + i) * kH + h) * kDv;
+        const float* op = o_part + (((long long)n * splits + i) * kH + h) * kDv + d0;
 #pragma unroll
-        for (int d = 0; d < kDv / 32; ++d) acc[d] = fmaf(wgt, op[d * 32 + lane], acc[d]);
+        for (int d = 0; d < kCombineDims / 32; ++d) acc[d] = fmaf(wgt, op[d * 32 + lane], acc[d]);
     }
-    __nv_bfloat16* ob = out + ((long long)n * kH + h) * kDv;
+    __nv_bfloat16* ob = out + ((long long)n * kH + h) * kDv + d0;
 #pragma unroll
-    for (int d = 0; d < kDv / 32; ++d) ob[d * 32 + lane] = __float2bfloat16_rn(acc[d]);
-    if (lse != nullptr && lane == 0)
+    for (int d = 0; d < kCombineDims / 32; ++d) ob[d * 32 + lane] = __float2bfloat16_rn(acc[d]);
+    if (lse != nullptr && lane == 0 && blockIdx.y == 0)
         lse[(long long)n * kH + h] = denom > 0.f ? mx + logf(denom) : -INFINITY;
 }
 
@@ -728,7 +735,8 @@ cudaError_t launch_sparse_mla_mma(const __nv_bfloat16* q, const void* kv, bool k
 
 cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int num_q, int splits,
                                __nv_bfloat16* out, float* lse, cudaStream_t stream) {
-    mla_combine_kernel<<<num_q, kH * 32, 0, stream>>>(o_part, lse_part, splits, out, lse);
+    mla_combine_kernel<<<dim3(num_q, kCombineParts), kH * 32, 0, stream>>>(o_part, lse_part, splits,
+                                                                          out, lse);
     count_launch(DSA_KERNEL_COMBINE);
     return cudaGetLastError();
 }
