@@ -12,8 +12,9 @@
 // consecutive TMEM columns that stay inside one thread -- no shuffles.
 //
 // Warp roles (640 threads): warp 0 issues TMA loads (query block once per unit, key tiles
-// through a ring of smem stages), warp 1 issues UMMAs into a ring of TMEM accumulators
-// (two of 256 columns in prefill), warp 2 owns the TMEM allocation, warps 4..19 drain the
+// through a ring of smem stages; for paged keys warps 2 and 3 issue the copies of two of
+// every three stages), warp 1 issues UMMAs into a ring of TMEM accumulators (two of 256
+// columns in prefill), warp 2 owns the TMEM allocation, warps 4..19 drain the
 // accumulators: tcgen05.ld, ReLU, weight, reduce, causal mask, coalesced fp32 stores.  The
 // drain is the longest stage per tile (16 max + 16 multiply-adds per score), so it gets
 // four warps per TMEM lane quadrant, each on a quarter of the block's queries, and the
@@ -48,6 +49,10 @@ constexpr uint32_t kTileBytes = kBM * 128;  // 128 keys x 64 bf16
 constexpr int kDecodeChunkTiles = 16;       // decode unit = 2048 keys
 constexpr int kPrefillChunkTiles = 32;      // prefill unit: at most 4096 keys
 constexpr int kPrefillQB = 16;              // prefill queries per block (UMMA N = 256)
+// Paged (decode) key tiles are copied by three producer warps (0, 2 and 3), each issuing
+// the copies of every third ring stage: one thread issuing TMA copies of 8 KB pages
+// reaches ~4.7 TB/s, whatever the number of copies in flight.
+constexpr int kDecodeProducers = 3;
 static_assert(kPrefillChunkTiles * 128 == 4096, "filtered candidate lists are per 4096-key chunk");
 
 template <int QB>
@@ -62,7 +67,8 @@ struct IdxSmem {
     uint64_t acc_full[4], acc_empty[4];
     uint32_t tmem_base;
     int abort;
-    int pages[kDecodeChunkTiles * kBM / 16];  // decode: the unit's page-table entries
+    int pages[kDecodeProducers][kDecodeChunkTiles * kBM / 16];  // decode: each producer's
+                                                                // copy of the unit's pages
 };
 
 // What the prefill epilogue does with each score.
@@ -165,27 +171,31 @@ __device__ __forceinline__ UnitInfo<QB, PAGED> unit_info(const IdxParams& p, int
     return x;
 }
 
-// One unit's copies, issued by the producer thread: the query block and its head weights
-// (once the previous user of the buffer is done), then every key tile into the ring.
-// Paged keys read their pool rows from sm.pages (filled by the producer warp).  Returns
+// One unit's copies, issued by a producer thread: the query block and its head weights
+// (producer 0, once the previous user of the buffer is done), then the key tiles of the
+// producer's ring stages (every stage in prefill; every kDecodeProducers-th, from stage
+// pw on, for paged keys, whose pool rows come from the producer's sm.pages[pw]).  Returns
 // false when a wait gave up.
 template <int QB, bool PAGED>
 __device__ __forceinline__ bool produce_unit(IdxSmem<QB>& sm, const IdxParams& p,
                                              const UnitInfo<QB, PAGED>& x, int ui, uint32_t& it,
                                              const CUtensorMap* tmap_q, const CUtensorMap* tmap_k,
-                                             volatile int* abort) {
+                                             volatile int* abort, int pw) {
     const int qb = ui & 1;
-    if (!mbar_wait(&sm.q_empty[qb], ((ui >> 1) & 1) ^ 1, abort, p.err)) return false;
-    // query block (TMA, swizzled) and its head weights (bulk copy) on one barrier
-    const int nq = PAGED ? 1 : x.len;
-    const uint32_t wbytes = (uint32_t)nq * kHI * 4;
-    mbar_arrive_expect_tx(&sm.q_full[qb], (uint32_t)(QB * kHI * 128) + wbytes);
-    tma_load_2d(sm.q[qb], tmap_q, 0, x.row0 * kHI, &sm.q_full[qb]);
-    bulk_load(sm.w[qb], p.w + (long long)x.row0 * kHI, wbytes, &sm.q_full[qb]);
+    if (pw == 0) {
+        if (!mbar_wait(&sm.q_empty[qb], ((ui >> 1) & 1) ^ 1, abort, p.err)) return false;
+        // query block (TMA, swizzled) and its head weights (bulk copy) on one barrier
+        const int nq = PAGED ? 1 : x.len;
+        const uint32_t wbytes = (uint32_t)nq * kHI * 4;
+        mbar_arrive_expect_tx(&sm.q_full[qb], (uint32_t)(QB * kHI * 128) + wbytes);
+        tma_load_2d(sm.q[qb], tmap_q, 0, x.row0 * kHI, &sm.q_full[qb]);
+        bulk_load(sm.w[qb], p.w + (long long)x.row0 * kHI, wbytes, &sm.q_full[qb]);
+    }
     for (int j = 0; j < x.ntiles; ++j, ++it) {
         constexpr int kStages = IdxSmem<QB>::kStages;
         const int st = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
+        if (PAGED && st % kDecodeProducers != pw) continue;
         if (!mbar_wait(&sm.k_empty[st], ph ^ 1, abort, p.err)) return false;
         const int tile = (x.tile0 + j) * (PAGED ? 1 : p.tile_stride);
         if constexpr (!PAGED) {
@@ -197,7 +207,7 @@ __device__ __forceinline__ bool produce_unit(IdxSmem<QB>& sm, const IdxParams& p
             const int used = min(per, (x.len - tile * kBM + ps - 1) / ps);
             mbar_arrive_expect_tx(&sm.k_full[st], (uint32_t)(used * ps * 128));
             for (int q = 0; q < used; ++q)
-                tma_load_2d(sm.k[st] + q * ps * 128, tmap_k, 0, sm.pages[j * per + q] * ps,
+                tma_load_2d(sm.k[st] + q * ps * 128, tmap_k, 0, sm.pages[pw][j * per + q] * ps,
                             &sm.k_full[st]);
         }
     }
@@ -255,8 +265,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0) {
-        // ---------------- TMA producer ----------------
+    if (warp == 0 || (PAGED && (warp == 2 || warp == 3))) {
+        // ---------------- TMA producer(s) ----------------
+        const int pw = warp == 0 ? 0 : warp - 1;  // paged keys: producers 0, 1, 2
         // Lane 0 issues the copies.  For paged keys the whole warp reads a unit's page-table
         // entries into shared memory first (one round trip per unit, not a dependent load
         // before every tile's copies), and the next unit's entries are loaded into
@@ -300,14 +311,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                             atomicOr(p.err, DSA_DEVERR_PAGE_RANGE);
                             pg = 0;
                         }
-                        sm.pages[q] = pg;
+                        sm.pages[pw][q] = pg;
                     }
                 }
                 __syncwarp();
                 load_pages(unit_at(i + 1), pg_next);
             }
             bool ok = true;
-            if (lane == 0) ok = produce_unit<QB, PAGED>(sm, p, x, ui, it, &tmap_q, &tmap_k, abort);
+            if (lane == 0) ok = produce_unit<QB, PAGED>(sm, p, x, ui, it, &tmap_q, &tmap_k, abort, pw);
             ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
             __syncwarp();  // lane 0 has issued every copy that reads sm.pages
             if (!ok) break;
