@@ -146,6 +146,19 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ------------------------------------------------------------------------------------
+// Programmatic dependent launch (griddepcontrol)
+// ------------------------------------------------------------------------------------
+// First statement of a kernel launched by launch_chained: waits until the grids this one
+// depends on have completed and their memory writes are visible (a no-op without the
+// launch attribute).  No kernel signals its dependents early: each CTA does so when it
+// exits, so the next kernel is launched while this one's last CTAs drain and its CTAs
+// take SMs as they free up.  (Signalling at the start of every CTA was measured slower:
+// the next kernel's waiting CTAs then hold SMs through the whole tail.)
+__device__ __forceinline__ void chained_launch_gate() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// ------------------------------------------------------------------------------------
 // tcgen05: TMEM allocation, MMA, commit, loads
 // ------------------------------------------------------------------------------------
 // Whole-warp call: allocates `ncols` TMEM columns and writes the base address to *dst.

@@ -233,6 +233,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     static_assert(!kSplitTiles || kAcc == 4, "tile turns need one accumulator per quarter");
 
     static_assert(MODE == kDense || !PAGED, "decode stores dense rows");
+    chained_launch_gate();
     if (p.guard != nullptr && *p.guard == 0) return;  // a fallback launch with nothing to do
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -509,9 +510,10 @@ cudaError_t launch_indexer_tc(const CUtensorMap& tq, const CUtensorMap& tk, cons
     cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<QB, PAGED, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    indexer_tc_kernel<QB, PAGED, MODE><<<grid, kThreads, smem, stream>>>(tq, tk, p);
+    e = launch_chained(indexer_tc_kernel<QB, PAGED, MODE>, dim3(grid), dim3(kThreads), smem, stream,
+                       1, tq, tk, p);
     count_launch(DSA_KERNEL_INDEXER);
-    return cudaGetLastError();
+    return e;
 }
 
 // Prefill launch of any mode: tensor maps, the unit count of the window and the grid.

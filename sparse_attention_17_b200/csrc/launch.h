@@ -24,6 +24,36 @@ cudaError_t get_dev_ctx(DevCtx* ctx);
 // Counts one launch of a kernel family (dsa_launch_count).
 void count_launch(int kind);
 
+// Launches a kernel whose first statement is chained_launch_gate() with programmatic
+// dependent launch allowed: it is launched once the previous kernel of the stream has no
+// CTA left running instead of once that kernel has completed, so that the launch overlaps
+// the completion; the gate keeps every global memory access after the previous work has
+// completed and is visible.  cluster > 1 adds a cluster dimension (x).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t stream, unsigned cluster, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // The calling thread's message for dsa_last_error: cleared on entry to every call, set
 // (printf-style) with the status a call returns on failure.
 void clear_last_error();

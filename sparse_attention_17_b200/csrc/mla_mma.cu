@@ -264,6 +264,7 @@ sparse_mla_mma_kernel(const Params p) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     volatile int* abort = &sm.abort;
+    chained_launch_gate();
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -620,6 +621,7 @@ constexpr int kCombineDims = kDv / kCombineParts;
 __global__ void __launch_bounds__(kH * 32)
 mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                    int splits, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+    chained_launch_gate();
     const int n = blockIdx.x;
     const int d0 = blockIdx.y * kCombineDims;
     const int h = threadIdx.x >> 5;
@@ -695,9 +697,9 @@ cudaError_t launch_mla_kernel(const Params& p, cudaStream_t stream, const DevCtx
     if (e != cudaSuccess) return e;
     const int slots = kCtasPerSm * ctx.num_sms;
     const int grid = p.num_units < slots ? p.num_units : slots;
-    sparse_mla_mma_kernel<kFp8><<<grid, kThreads, smem, stream>>>(p);
+    e = launch_chained(sparse_mla_mma_kernel<kFp8>, dim3(grid), dim3(kThreads), smem, stream, 1, p);
     count_launch(DSA_KERNEL_ATTENTION);
-    return cudaGetLastError();
+    return e;
 }
 }  // namespace
 
@@ -735,10 +737,11 @@ cudaError_t launch_sparse_mla_mma(const __nv_bfloat16* q, const void* kv, bool k
 
 cudaError_t launch_mla_combine(const float* o_part, const float* lse_part, int num_q, int splits,
                                __nv_bfloat16* out, float* lse, cudaStream_t stream) {
-    mla_combine_kernel<<<dim3(num_q, kCombineParts), kH * 32, 0, stream>>>(o_part, lse_part, splits,
-                                                                          out, lse);
+    const cudaError_t e = launch_chained(mla_combine_kernel, dim3(num_q, kCombineParts),
+                                         dim3(kH * 32), 0, stream, 1, o_part, lse_part, splits,
+                                         out, lse);
     count_launch(DSA_KERNEL_COMBINE);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace dsa

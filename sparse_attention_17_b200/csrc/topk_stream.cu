@@ -479,6 +479,7 @@ topk_stream_kernel(const float* __restrict__ scores, long long ld, int rows, int
                    const int* __restrict__ row_len, int max_len, int k, int* __restrict__ idx,
                    long long ld_idx, const int* __restrict__ row_mask, int idx_offset,
                    unsigned* __restrict__ err) {
+    chained_launch_gate();
     extern __shared__ __align__(16) unsigned char smem_raw[];
     StreamSmem& sm = *reinterpret_cast<StreamSmem*>(smem_raw);
     const int max_chunks = (max_len + kChunk - 1) / kChunk;
@@ -528,6 +529,7 @@ topk_cluster_kernel(const float* __restrict__ scores, long long ld, int rows, in
                     long long ld_idx, const int* __restrict__ row_mask, int idx_offset,
                     unsigned* __restrict__ err) {
     namespace cg = cooperative_groups;
+    chained_launch_gate();
     extern __shared__ __align__(16) unsigned char smem_raw[];
     StreamSmem& sm = *reinterpret_cast<StreamSmem*>(smem_raw);
     const int max_chunks = (max_len + kChunk - 1) / kChunk;
@@ -605,10 +607,10 @@ cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
-        kernel<<<rows, 256, smem, stream>>>(scores, ld, rows, q_begin, row_len, max_len, k, idx,
-                                            ld_idx, row_mask, idx_offset, ctx.err);
+        e = launch_chained(kernel, dim3(rows), dim3(256), smem, stream, 1, scores, ld, rows, q_begin,
+                           row_len, max_len, k, idx, ld_idx, row_mask, idx_offset, ctx.err);
         count_launch(DSA_KERNEL_TOPK);
-        return cudaGetLastError();
+        return e;
     }
     // At most half as many rows as SMs (a decode batch): a pair of 512-thread CTAs per row
     // (a cluster of two), which halves the candidate pass of each row and keeps the
@@ -622,20 +624,9 @@ cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(rows * cl));
-        cfg.blockDim = dim3(kClusterThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)cl;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, kernel, scores, ld, rows, q_begin, row_len, max_len, k, idx,
-                               ld_idx, row_mask, idx_offset, ctx.err);
+        e = launch_chained(kernel, dim3((unsigned)(rows * cl)), dim3(kClusterThreads), smem, stream,
+                           (unsigned)cl, scores, ld, rows, q_begin, row_len, max_len, k, idx,
+                           ld_idx, row_mask, idx_offset, ctx.err);
         count_launch(DSA_KERNEL_TOPK);
         return e;
     }
@@ -643,10 +634,10 @@ cudaError_t launch_topk(const float* scores, long long ld, int rows, int q_begin
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    kernel<<<rows, 1024, smem, stream>>>(scores, ld, rows, q_begin, row_len, max_len, k, idx,
-                                         ld_idx, row_mask, idx_offset, ctx.err);
+    e = launch_chained(kernel, dim3(rows), dim3(1024), smem, stream, 1, scores, ld, rows, q_begin,
+                       row_len, max_len, k, idx, ld_idx, row_mask, idx_offset, ctx.err);
     count_launch(DSA_KERNEL_TOPK);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace dsa
