@@ -358,6 +358,8 @@ def run_native(args, rank, world, local_rank):
     # i-1's download overlap the computation of the step in between.
     e2e = None
     if not args.no_e2e:
+        # the device-resident run's output, to check the pipelined steps against
+        ref_out = out.cpu()
         pinned = {n: host[n].pin_memory() for n in names}
         h2d = sum(t.numel() * t.element_size() for t in pinned.values())
         xs = [x, {n: torch.empty_like(x[n]) for n in names}]
@@ -417,6 +419,10 @@ def run_native(args, rank, world, local_rank):
         t2.record(stream)
         torch.cuda.synchronize()
         e2e_ms = s2.elapsed_time(t2) / n_e2e
+        # the last two steps' outputs, read back through the pipeline, are the device run's
+        outputs_match = all(torch.equal(out_host[b].view(torch.int16), ref_out.view(torch.int16))
+                            for b in range(2))
+        del ref_out
         e2e_ms = max_over_ranks(e2e_ms, dev)
 
         # the copies alone, each direction on its own stream: the host link's bound on e2e
@@ -472,7 +478,8 @@ def run_native(args, rank, world, local_rank):
                "h2d_gbs_alone": round(h2d / (h2d_ms / 1e3) / 1e9, 1),
                "d2h_gbs_alone": round(d2h / (d2h_ms / 1e3) / 1e9, 1),
                "copy_bound_ms": round(max(h2d_ms, d2h_ms), 3),
-               "copy_both_directions_ms": round(both_ms, 3)}
+               "copy_both_directions_ms": round(both_ms, 3),
+               "outputs_match_device_run": outputs_match}
 
     result = None
     if rank == 0:
