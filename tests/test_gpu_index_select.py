@@ -99,6 +99,21 @@ def test_misleading_sample_falls_back_to_dense():
     assert torch.equal(a, b)
 
 
+def test_misleading_sample_in_narrow_windows():
+    """The same planted keys with 64-row windows: each window's fallback top-k is a launch
+    of few rows, which takes the cluster path (two CTAs per row) with a row mask."""
+    T, k = 12288, 2048
+    d = G.indexer_gauss(T, 10)
+    s = torch.arange(T)
+    sampled = (s // 128) % 16 == 0
+    d["k_idx"][sampled] = (d["k_idx"][sampled].float() * 4).to(torch.bfloat16)
+    q_idx, k_idx, w = _cuda(d)
+    q_begin, rows = T - 256, 256
+    a = _fused(q_idx, k_idx, w, k, q_begin, rows, window=64)
+    b = _dense(q_idx, k_idx, w, k, q_begin, rows)
+    assert torch.equal(a, b)
+
+
 def test_against_oracle_sampled_rows():
     """T=12000 integer inputs, rows past the no-sample bound checked against the oracle."""
     T, k = 12000, 2048
