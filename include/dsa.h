@@ -31,7 +31,11 @@
  *   - Tensors are dense row-major ("C order") unless a leading dimension is given.
  *     Tensor pointers must be 16-byte aligned; leading dimensions are in elements.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
- *     stream).  Results are valid once the stream has reached the call.
+ *     stream).  Results are valid once the stream has reached the call.  The indexer,
+ *     top-k, attention and split-merge kernels are launched with programmatic dependent
+ *     launch: one may start while the previous kernel of the stream drains, and waits
+ *     (griddepcontrol) for that work to complete before touching memory, so stream order
+ *     holds as for any launch.
  *   - Argument errors return DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED before anything is
  *     launched; dsa_last_error() then describes the problem.  DSA_ERR_CUDA reports a
  *     failed launch or CUDA runtime call.
