@@ -34,7 +34,8 @@
 //           selected key its output position: ascending order without sorting.
 // Rows whose candidates number fewer than k or more than the buffer holds (a sample that
 // misled, heavy ties) are redone exactly from global memory: four 8-bit radix passes over
-// the row for tau and need, then one ordered pass with a block scan per 1024 keys.
+// the row for tau and need, then one ordered pass with a block scan per four keys of every
+// thread.
 #include <cooperative_groups.h>
 
 #include "dsa_common.cuh"
