@@ -269,10 +269,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
     if (warp == 0 || (PAGED && (warp == 2 || warp == 3))) {
         // ---------------- TMA producer(s) ----------------
         const int pw = warp == 0 ? 0 : warp - 1;  // paged keys: producers 0, 1, 2
-        // Lane 0 issues the copies.  For paged keys the whole warp reads a unit's page-table
-        // entries into shared memory first (one round trip per unit, not a dependent load
-        // before every tile's copies), and the next unit's entries are loaded into
-        // registers while lane 0 issues this unit's copies, so that round trip overlaps them.
+        // Lane 0 issues the copies.  For paged keys each producer warp reads a unit's
+        // page-table entries into its own shared copy first (one round trip per unit, not a
+        // dependent load before every tile's copies), and the next unit's entries are
+        // loaded into registers while lane 0 issues this unit's copies, so that round trip
+        // overlaps them.
         if (lane == 0) {
             tma_prefetch_desc(&tmap_q);
             tma_prefetch_desc(&tmap_k);
